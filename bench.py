@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA decode step (indexer -> top-k -> sparse MLA) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode32k]
+    python bench.py --impl reference ...        # the fp64 CPU oracle arm
+
+One step = one pass of the whole hot path over one batch of the workload
+(decode32k: one 32K-context sequence; batched: 32 ragged sequences; fp8: 4
+sequences at 128K with an e4m3 indexer cache).  Inputs are seeded synthetic
+data drawn on the device; the timed region replays CUDA graphs that hold
+exactly K steps, each step reading its own copy of the caches (copies rotate
+over more than 3x the L2 size, so every step starts with a cold L2).
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+replica (the path shards by sequence and has no exchange step), the timed
+region is bracketed by barriers and the max over ranks is used.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DSA decode steps/s @32K ctx (indexer+top-k+sparse MLA); % HBM roofline"
+UNIT = "steps/s"
+L2_BYTES_DEFAULT = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def stage_bytes(wl, end_pos):
+    """Algorithmic HBM bytes per step, per stage and for the whole step.
+
+    Only what the method must move: the indexer key cache (+ e4m3 scales),
+    q_I and w, the selected latent rows (576 bf16 each), q and the output.
+    Scores and indices are intermediates; the per-stage figures include the
+    stage's own output so that each kernel's roofline is stated on what it
+    must write."""
+    H, k = wl.H, wl.topk
+    fp8 = wl.idx_dtype == "e4m3"
+    key_row = 128 + 4 if fp8 else 256
+    qi = 64 * 128 * (1 if fp8 else 2)
+    out_b = 4 if wl.out_dtype == "f32" else 2
+    T = wl.T
+    idx = topk_b = mla = step = 0
+    for E in end_pos:
+        valid_sum = sum(min(E, E - T + t + 1) for t in range(T))
+        keff_sum = sum(min(k, E - T + t + 1) for t in range(T))
+        idx += E * key_row + T * (qi + 256) + valid_sum * 4
+        topk_b += valid_sum * 4 + T * k * 4
+        mla += keff_sum * 1152 + T * H * (576 * 2 + 512 * out_b)
+        step += E * key_row + T * (qi + 256) + keff_sum * 1152 + T * H * (576 * 2 + 512 * out_b)
+    return {"indexer": idx, "topk": topk_b, "sparse_mla": mla, "step": step}
+
+
+def oracle_work(wl, end_pos):
+    """Multiply-adds of one oracle step (indexer 64*128 per key, MLA H*(576+512) per kept key)."""
+    T = wl.T
+    w = 0
+    for E in end_pos:
+        for t in range(T):
+            L = E - T + t + 1
+            w += L * 8192 + min(wl.topk, L) * wl.H * 1088
+    return w
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a host float over ranks (identity when world == 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(steps_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank's steps over the slowest rank's time."""
+    return steps_per_rank * world / max_seconds
+
+
+# ---------------------------------------------------------------- CPU (oracle) timing
+
+def oracle_step_inputs(wl, inp_cpu, budget_work):
+    """A bounded sample of one step for the oracle: whole sequences while they
+    fit the budget, else a prefix of one sequence's keys (topk and kept rows
+    scaled with it).  Returns (sample Inputs, fraction of the full step's work)."""
+    from sparse_attention_04_b200 import inputs as I
+    full = oracle_work(wl, inp_cpu.end_pos)
+    seqs, acc = [], 0
+    for b, E in enumerate(inp_cpu.end_pos):
+        wk = oracle_work(wl, [E])
+        if acc + wk > budget_work and seqs:
+            break
+        seqs.append(b)
+        acc += wk
+    if acc <= budget_work:
+        eps = [inp_cpu.end_pos[b] for b in seqs]
+        sub_wl = I.Workload(wl.name, len(seqs), wl.T, None, None, wl.topk, wl.H, wl.idx_dtype, wl.scale,
+                            wl.out_dtype, wl.seed)
+        return _slice(inp_cpu, sub_wl, seqs, eps), acc / full
+    # one sequence is already over budget: keep a prefix of m-th of its keys
+    E = inp_cpu.end_pos[0]
+    m = max(1, math.ceil(oracle_work(wl, [E]) / budget_work))
+    E2 = max(wl.T, E // m)
+    k2 = max(1, wl.topk // m)
+    sub_wl = I.Workload(wl.name, 1, wl.T, None, None, k2, wl.H, wl.idx_dtype, wl.scale, wl.out_dtype, wl.seed)
+    sub = _slice(inp_cpu, sub_wl, [0], [E2])
+    return sub, oracle_work(sub_wl, [E2]) / full
+
+
+def _slice(inp, wl, seqs, eps):
+    import torch
+    from sparse_attention_04_b200.inputs import Inputs
+    off = inp.offsets.tolist()
+    cat = lambda t: torch.cat([t[off[b]:off[b] + e] for b, e in zip(seqs, eps)]).contiguous()
+    new_off = [0]
+    for e in eps:
+        new_off.append(new_off[-1] + e)
+    ks = None if inp.k_scale is None else cat(inp.k_scale)
+    # the T query rows of a truncated sequence are its last T positions
+    return Inputs(wl, eps, torch.tensor(new_off, dtype=torch.int32), inp.q_idx[seqs].contiguous(),
+                  inp.w[seqs].contiguous(), cat(inp.k_idx), ks, inp.q[seqs].contiguous(), cat(inp.kv))
+
+
+def time_oracle(wl, inp_cpu, n_steps, seconds_per_step_budget):
+    """Runs n_steps oracle steps on a bounded sample; returns (full steps/s, cores, sample text)."""
+    import oracle
+    # calibrate the oracle's multiply-add rate on a small slice
+    probe_wl_inp, frac0 = oracle_step_inputs(wl, inp_cpu, 2e8)
+    t0 = time.perf_counter()
+    oracle.decode_step(probe_wl_inp)
+    rate = oracle_work(probe_wl_inp.wl, probe_wl_inp.end_pos) / max(time.perf_counter() - t0, 1e-6)
+    sample, frac = oracle_step_inputs(wl, inp_cpu, max(1e6, rate * seconds_per_step_budget))
+    t0 = time.perf_counter()
+    for _ in range(n_steps):
+        oracle.decode_step(sample)
+    dt = time.perf_counter() - t0
+    per_full_step = dt / n_steps / frac
+    text = (f"{n_steps} oracle step(s) on {len(sample.end_pos)} sequence(s) with end_pos {sample.end_pos[:4]}"
+            f"{'...' if len(sample.end_pos) > 4 else ''}, topk {sample.wl.topk}; time scaled by "
+            f"{1 / frac:.2f} (multiply-add count of the full step / the sample's)")
+    return 1.0 / per_full_step, oracle.num_threads(), text
+
+
+# ---------------------------------------------------------------- native arm
+
+def run_native(args, rank, world, local):
+    import torch
+    from sparse_attention_04_b200 import _lib, api
+    from sparse_attention_04_b200 import inputs as I
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = I.WORKLOADS[args.workload]
+    if wl.T != 1:
+        raise SystemExit("bench times decode workloads (T = 1)")
+    base = I.make_inputs(wl, dev)
+    E = base.end_pos
+    max_e = max(E)
+    sb = stage_bytes(wl, E)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size or L2_BYTES_DEFAULT
+    n_copies = max(2, math.ceil(3 * l2 / sb["step"]))
+    per_copy = sum(t.numel() * t.element_size() for t in
+                   (base.k_idx, base.kv, base.q_idx, base.w, base.q) + ((base.k_scale,) if base.k_scale is not None else ()))
+    free, _ = torch.cuda.mem_get_info(dev)
+    n_copies = max(2, min(n_copies, int(0.5 * free // per_copy)))
+    clone = lambda t: None if t is None else t.clone()
+    copies = [base] + [I.Inputs(wl, E, base.offsets, clone(base.q_idx), clone(base.w), clone(base.k_idx),
+                                clone(base.k_scale), clone(base.q), clone(base.kv)) for _ in range(n_copies - 1)]
+    step = api.DecodeStep(wl.B, max_e, wl.topk, wl.H,
+                          torch.float32 if wl.out_dtype == "f32" else torch.bfloat16, dev)
+    rows = base.rows
+
+    def one_step(c):
+        x = copies[c % n_copies]
+        step(x.q_idx, x.w, x.k_idx, x.k_scale, x.q, x.kv, x.offsets, rows, wl.scale)
+
+    one_step(0)
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise SystemExit("device status " + _lib.status_string(int(step.status.item())))
+
+    K, W = args.steps, args.warmup
+    G = min(K, args.graph_steps)
+    stream = torch.cuda.Stream(dev)
+
+    def capture(n, start):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                one_step(start + i)
+        return g
+
+    graph_main = capture(G, 0)
+    graph_rem = capture(K % G, 0) if K % G else None
+    graph_warm = capture(min(W, G), 0) if W > 0 else None
+    launches_per_step = 3 + (1 if _lib.sparse_mla_workspace_size(wl.B, 1, wl.H, wl.topk) > 0 else 0)
+
+    # ---- warm-up (untimed)
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(max(1, W // max(1, min(W, G)))):
+        if graph_warm is not None:
+            graph_warm.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(K // G):
+            graph_main.replay()
+        if graph_rem is not None:
+            graph_rem.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    elapsed = ev0.elapsed_time(ev1) / 1e3
+    t_max = reduce_max(elapsed, world, dev)
+    value = aggregate_value(K, world, t_max)
+    ms_per_step = t_max / K * 1e3
+
+    # ---- per-stage durations (same kernels, events between stages, in a graph)
+    n_prof = min(64, max(8, K))
+    ld = step.ld
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
+    ws_mla = step.workspace[_lib.decode_step_workspace_layout(wl.B, max_e, wl.topk, wl.H)[3]:]
+    g_prof = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_prof, stream=stream):
+        for i in range(n_prof):
+            x = copies[i % n_copies]
+            evs[i][0].record()
+            _lib.indexer_scores(x.q_idx, x.w, x.k_idx, x.k_scale, x.offsets, wl.B, 1, rows, step.scores, ld,
+                                status=step.status)
+            evs[i][1].record()
+            _lib.topk(step.scores, ld, x.offsets, wl.B, 1, wl.topk, step.indices, status=step.status)
+            evs[i][2].record()
+            _lib.sparse_mla(x.q, x.kv, x.offsets, step.indices, wl.B, 1, wl.H, wl.topk, wl.scale, rows,
+                            step.out, lse=step.lse, workspace=ws_mla, status=step.status)
+            evs[i][3].record()
+    g_prof.replay()
+    g_prof.replay()
+    torch.cuda.synchronize()
+    names = ["indexer", "topk", "sparse_mla"]
+    stage_s = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_prof)) / n_prof / 1e3
+               for j, n in enumerate(names)}
+    dominant = max(stage_s, key=stage_s.get)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    except Exception:
+        hbm_peak, peak_src = 6650.0, "fallback"
+    achieved = sb[dominant] / stage_s[dominant] / 1e9
+    traffic = load_traffic(args.workload, dominant)
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "peak_source": peak_src,
+                "stage_us": {n: round(v * 1e6, 3) for n, v in stage_s.items()},
+                "stage_frac": {n: round(sb[n] / stage_s[n] / 1e9 / hbm_peak, 4) for n in names},
+                "step_frac": round(sb["step"] * (value / world) / 1e9 / hbm_peak, 4)}
+
+    # ---- end to end: host buffers in, host result out, through the C ABI
+    e2e = run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world)
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if wl.idx_dtype == "bf16" else "e4m3+bf16",
+            "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
+            "config": {"workload": args.workload, "B": wl.B, "end_pos": E if len(E) <= 4 else
+                       {"min": min(E), "max": max(E), "sum": sum(E)}, "topk": wl.topk, "heads": wl.H,
+                       "indexer": f"64x128 {wl.idx_dtype}", "parallelism": f"replicas x{world}",
+                       "l2": f"cold: {n_copies} rotating cache copies (> 3x L2)",
+                       "algorithmic_bytes_per_step": sb["step"]},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * K, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = base.to("cpu")
+        v, cores, text = time_oracle(wl, cpu, n_steps=3, seconds_per_step_budget=args.cpu_seconds / 3)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": text}
+    if world > 1:
+        import torch.distributed as dist
+        del g_prof, graph_main, graph_rem, graph_warm
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world):
+    """Per step: host->device copy of the new token's inputs (q_I, w, q and
+    the new key / latent rows, written over the cache's last row), the decode
+    step, device->host copy of the output.  Pinned host buffers, one CUDA graph."""
+    import torch
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+    x0 = copies[0]
+    last = x0.offsets[1:].cpu().long() - 1  # last cache row of every sequence
+    h_qi, h_w, h_q = pin(x0.q_idx), pin(x0.w), pin(x0.q)
+    h_k, h_kv = pin(x0.k_idx[last]), pin(x0.kv[last])
+    h_ks = None if x0.k_scale is None else pin(x0.k_scale[last])
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
+    last_d = last.to(dev)
+    d_k_row = torch.empty_like(x0.k_idx[last])
+    d_kv_row = torch.empty_like(x0.kv[last])
+    nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
+    h2d = sum(nbytes(t) for t in (h_qi, h_w, h_q, h_k, h_kv, h_ks))
+    d2h = nbytes(h_out)
+
+    def e2e_step(i):
+        x = copies[i % n_copies]
+        x.q_idx.copy_(h_qi, non_blocking=True)
+        x.w.copy_(h_w, non_blocking=True)
+        x.q.copy_(h_q, non_blocking=True)
+        d_k_row.copy_(h_k, non_blocking=True)
+        d_kv_row.copy_(h_kv, non_blocking=True)
+        x.k_idx.index_copy_(0, last_d, d_k_row)
+        x.kv.index_copy_(0, last_d, d_kv_row)
+        if h_ks is not None:
+            x.k_scale.index_copy_(0, last_d, h_ks.to(dev, non_blocking=True))
+        step(x.q_idx, x.w, x.k_idx, x.k_scale, x.q, x.kv, x.offsets, x.rows, wl.scale)
+        h_out.copy_(step.out, non_blocking=True)
+
+    Ge = min(G, 256)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(Ge):
+            e2e_step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, K // Ge)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t = reduce_max(ev0.elapsed_time(ev1) / 1e3, world, dev)
+    return {"value": round(aggregate_value(reps * Ge, world, t), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "caches stay resident; per step the new token's q_I, w, q, key row and latent row go in, the output comes out"}
+
+
+def load_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary for this kernel and
+    workload, if one exists for the current kernel version; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        return d.get(workload, {}).get(kernel)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The fp64 oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from sparse_attention_04_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload]
+    inp = I.make_inputs(wl, "cpu")
+    budget = max(0.002, args.reference_seconds / max(1, args.steps + args.warmup))
+    import oracle
+    sample, frac = oracle_step_inputs(wl, inp, 1e6)
+    # calibrate, then size the per-step sample to the budget
+    t0 = time.perf_counter()
+    oracle.decode_step(sample)
+    rate = oracle_work(sample.wl, sample.end_pos) / max(time.perf_counter() - t0, 1e-6)
+    sample, frac = oracle_step_inputs(wl, inp, max(1e5, rate * budget))
+    for _ in range(args.warmup):
+        oracle.decode_step(sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_step(sample)
+    dt = time.perf_counter() - t0
+    value = args.steps * frac / dt
+    text = (f"each step: the oracle on {len(sample.end_pos)} sequence(s), end_pos {sample.end_pos[:4]}, "
+            f"topk {sample.wl.topk}; scaled by {1 / frac:.2f} (multiply-add count of the full step / the sample's)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1))", "config": {"workload": args.workload, "B": wl.B,
+                                                           "topk": wl.topk, "heads": wl.H},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": text},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "batched", "fp8", "tiny"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--graph-steps", type=int, default=500)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    if world != args.gpus and world != 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_native(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The path has three stages, each a call below, plus one call that runs all
+ * three for a decode step:
+ *
+ *   1. dsa_indexer_scores  lightning-indexer scores with the causal mask
+ *        I[t,s] = sum_h w[t,h] * ReLU(q_I[t,h,:] . k_I[s,:])
+ *      ("DeepSeek-V3.2-Exp - Keep top-k positions", Indexer.forward listing,
+ *       the fp8_index call and "index_score += mask"; the head sum is the fix
+ *       in "[WIP] deepseek v32", mlx-lm PR #512).
+ *   2. dsa_topk  keep each query's min(k, valid) highest-scoring positions
+ *      (same page, the M^sel formula and "topk(min(index_topk, end_pos))").
+ *   3. dsa_sparse_mla  absorbed MLA over only the selected latent rows
+ *      ("DeepSeek-V3.2-Exp - Apply sparse mask", MQA decode listing:
+ *       scores = q.[kv||pe] * scale, the -inf index mask, softmax, P.kv).
+ *
+ * Shapes and layouts (all device pointers, row-major, no padding unless said):
+ *   H_I = 64 indexer heads, D_I = 128 indexer dim, D_QK = 576 (512 latent ||
+ *   64 rope), D_V = 512, H = MLA heads (1..128).
+ *   offsets  int32 [B+1], device.  Sequence b owns rows [offsets[b],
+ *            offsets[b+1]) of BOTH caches; end_pos_b = offsets[b+1]-offsets[b].
+ *            Its T query rows sit at absolute positions end_pos_b - T + t.
+ *   kv_rows  number of rows the caches were allocated with (>= offsets[B]);
+ *            bounds every cache read.
+ *   q_idx    [B,T,64,128] bf16, or e4m3 codes (uint8) when idx_dtype=DSA_E4M3
+ *   w        [B,T,64] fp32 per-head weights; for e4m3 the per-(t,h) q scale
+ *            is already multiplied in, as the listing does before fp8_index
+ *   k_idx    [kv_rows,128] bf16 or e4m3 codes;  k_scale [kv_rows] fp32 (e4m3 only)
+ *   scores   fp32, row (b,t) starts at scores + (b*T+t)*ld_scores
+ *   indices  int32 [B,T,k], sequence-local positions, ascending, -1 padded
+ *   q        [B,T,H,576] bf16 absorbed query;  kv [kv_rows,576] bf16
+ *   out      [B,T,H,512] bf16 or fp32;  lse [B,T,H] fp32 natural-log, optional
+ *
+ * Ownership and errors.  The caller allocates and owns every buffer, the
+ * workspace included; the library allocates nothing and keeps no state between
+ * calls.  Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream).  Argument errors are returned before anything is
+ * launched.  A launch failure returns DSA_ERR_CUDA.  Problems only the device
+ * can see (offsets that break the bounds above, an index outside [0,end_pos),
+ * a pipeline wait that ran out of time) are written as a DSA status code into
+ * *dev_status (device int32, optional, never cleared by the library) and the
+ * affected row is skipped or zeroed; read it after synchronising.
+ * Device pointers must be 16-byte aligned.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or enum       */
+  DSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. H > 128)  */
+  DSA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required   */
+  DSA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed         */
+  DSA_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran out of time   */
+  DSA_ERR_BAD_INDEX = 6,   /* device: an index outside [0, end_pos)     */
+  DSA_ERR_BAD_OFFSETS = 7  /* device: offsets exceed kv_rows / ld / T   */
+} dsa_status_t;
+
+enum { DSA_BF16 = 0, DSA_E4M3 = 1, DSA_F32 = 2 };
+
+/* Largest k accepted by dsa_topk / dsa_sparse_mla (index_topk = 2048). */
+#define DSA_MAX_TOPK 2048
+/* Largest MLA head count (the 128 heads of the decode listing). */
+#define DSA_MAX_HEADS 128
+
+/* Human-readable name of a status code; never NULL. */
+const char* dsa_status_string(int status);
+
+/* ABI version of this library (major*100 + minor). */
+int dsa_version(void);
+
+/*
+ * Stage 1 -- indexer scores ("Keep top-k positions", Indexer.forward: the
+ * fp8_index call over k_cache[:end_pos] and "index_score += mask").
+ * Writes, for every row (b,t) and every s < end_pos_b:
+ *   scores[(b*T+t)*ld_scores + s] = s <= end_pos_b-T+t
+ *       ? sum_h w[b,t,h] * ReLU(q_I[b,t,h,:] . k_I[offsets[b]+s,:]) (* k_scale for e4m3)
+ *       : -inf
+ * Entries at s >= end_pos_b are not touched.  ld_scores >= max end_pos, a
+ * multiple of 4.  Bytes read: the key cache once, q_I and w once.
+ */
+int dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+                       const float* k_scale, int idx_dtype, const int32_t* offsets,
+                       int B, int T, int64_t kv_rows, float* scores, int64_t ld_scores,
+                       int32_t* dev_status, void* stream);
+
+/*
+ * Stage 2 -- top-k ("Keep top-k positions": topk(min(index_topk, end_pos))
+ * and M^sel).  For row (b,t) the valid positions are s < min(end_pos_b,
+ * end_pos_b-T+t+1) (the causal prefix); it keeps k_eff = min(k, #valid) of
+ * them, ordered by larger score first and then lower position (-0.0 == +0.0),
+ * and writes them ascending into indices[(b*T+t)*k ...], then -1 up to k.
+ * Deterministic: the same scores always give the same indices.  1 <= k <= 2048.
+ */
+int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* offsets, int B, int T,
+             int k, int32_t* indices, int32_t* dev_status, void* stream);
+
+/*
+ * Stage 3 -- sparse absorbed MLA ("Apply sparse mask", MQA decode listing).
+ * For each row r=(b,t), head h, the selected positions j (indices >= 0):
+ *   l_j = scale * q[r,h,:576] . kv[offsets[b]+j, :576];  p = softmax_j(l)
+ *   out[r,h,:] = sum_j p_j * kv[offsets[b]+j, :512];  lse[r,h] = log sum_j exp(l_j)
+ * Rows with no selected position get out = 0, lse = -inf.  Indices outside
+ * [0,end_pos_b) are treated as empty and reported as DSA_ERR_BAD_INDEX.
+ * workspace: dsa_sparse_mla_workspace_size(B,T,H,k) bytes (may be 0 -> NULL ok).
+ */
+size_t dsa_sparse_mla_workspace_size(int B, int T, int H, int k);
+int dsa_sparse_mla(const void* q, const void* kv, const int32_t* offsets, const int32_t* indices,
+                   int B, int T, int H, int k, float scale, int64_t kv_rows, void* out,
+                   int out_dtype, float* lse, void* workspace, size_t ws_bytes,
+                   int32_t* dev_status, void* stream);
+
+/*
+ * The whole decode step (T = 1): stages 1 -> 2 -> 3 on `stream`, scores and
+ * indices kept in the workspace.  max_end_pos bounds every end_pos_b (it sets
+ * the workspace's score pitch).  Same layouts as above with T = 1.
+ * workspace: dsa_decode_step_workspace_size(B, max_end_pos, k, H) bytes.
+ */
+size_t dsa_decode_step_workspace_size(int B, int max_end_pos, int k, int H);
+int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
+                    int idx_dtype, const void* q, const void* kv, const int32_t* offsets, int B,
+                    int max_end_pos, int64_t kv_rows, int k, int H, float scale, void* out,
+                    int out_dtype, float* lse, void* workspace, size_t ws_bytes,
+                    int32_t* dev_status, void* stream);
+
+/*
+ * Where, inside a decode-step workspace, the step leaves its intermediates
+ * (byte offsets; the scores pitch is returned in *ld_scores).  For tests and
+ * tools that want to look at stage outputs; the layout may change between
+ * versions.
+ */
+int dsa_decode_step_workspace_layout(int B, int max_end_pos, int k, int H, size_t* scores_off,
+                                     int64_t* ld_scores, size_t* indices_off, size_t* mla_off);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

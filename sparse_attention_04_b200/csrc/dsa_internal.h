@@ -1,0 +1,78 @@
+// dsa_internal.h -- constants and launcher declarations shared by the kernel
+// translation units and the C-ABI layer (dsa_api.cu).  Not installed.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+constexpr int kHI = 64;    // indexer heads
+constexpr int kDI = 128;   // indexer head dim
+constexpr int kDQK = 576;  // latent 512 || rope 64
+constexpr int kDV = 512;   // value width (the latent)
+constexpr int kMaxTopk = DSA_MAX_TOPK;
+constexpr int kMaxHeads = DSA_MAX_HEADS;
+
+// Every pipeline wait in the kernels gives up after this long and reports
+// DSA_ERR_TIMEOUT.  Normal waits last microseconds.
+constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;
+
+// Per-device facts the launchers need (cached after the first query).
+struct DeviceInfo {
+  int sm_count;
+  int max_smem_optin;
+};
+const DeviceInfo& device_info();
+
+// ---- stage 1: indexer ------------------------------------------------------
+struct IndexerArgs {
+  const void* q_idx;
+  const float* w;
+  const void* k_idx;
+  const float* k_scale;
+  int idx_dtype;
+  const int32_t* offsets;
+  int B, T;
+  int64_t kv_rows;
+  float* scores;
+  int64_t ld;
+  int32_t* status;
+};
+int launch_indexer(const IndexerArgs& a, cudaStream_t stream);
+
+// ---- stage 2: top-k ---------------------------------------------------------
+struct TopkArgs {
+  const float* scores;
+  int64_t ld;
+  const int32_t* offsets;
+  int B, T, k;
+  int32_t* indices;
+  int32_t* status;
+};
+int launch_topk(const TopkArgs& a, cudaStream_t stream);
+
+// ---- stage 3: sparse MLA ----------------------------------------------------
+struct MlaArgs {
+  const void* q;
+  const void* kv;
+  const int32_t* offsets;
+  const int32_t* indices;
+  int B, T, H, k;
+  float scale;
+  int64_t kv_rows;
+  void* out;
+  int out_dtype;
+  float* lse;
+  void* workspace;
+  size_t ws_bytes;
+  int32_t* status;
+};
+int mla_num_splits(int n_rows, int k);
+size_t mla_workspace_bytes(int n_rows, int H, int k);
+int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,377 @@
+// indexer.cu -- stage 1: lightning-indexer scores on the tcgen05 tensor core.
+//
+// I[t,s] = sum_h w[t,h] * ReLU(q_I[t,h,:] . k_I[s,:])  (+ causal mask)
+// ("DeepSeek-V3.2-Exp - Keep top-k positions", Indexer.forward: the fp8_index
+// call and "index_score += mask"; the sum over heads is the fix of
+// "[WIP] deepseek v32", mlx-lm PR #512.)
+//
+// Orientation: keys on the MMA's M (128 TMEM lanes), (query, head) pairs on N.
+// One tile = 128 keys x NQ queries x 64 heads, K = 128:
+//     D[key, q*64+h] = k_I[key,:] . q_I[q,h,:]
+// so every epilogue thread owns one key (one TMEM lane) and forms
+// sum_h w * max(0, D) from its own registers -- no cross-lane reduction.
+//
+// Roles (one CTA per SM, persistent over a balanced range of a flat list of
+// (sequence, query block, key tile) items):
+//   warps 0-3  epilogue: TMEM -> registers, ReLU, weight, head sum, mask, store
+//   warp  4    TMA producer: key tiles into a ring of stages, query blocks
+//              into two slots (reloaded only when the query block changes)
+//   warp  5    TMEM allocator + MMA issuer (one thread)
+// Key tiles and query blocks land in shared memory in the 128-byte-swizzled
+// K-major layout the MMA descriptors describe; accumulators are double
+// buffered in TMEM so the epilogue of tile i overlaps the MMA of tile i+1.
+#include <cuda.h>
+
+#include "dsa_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace dsa {
+namespace {
+
+template <int NQ, bool FP8>
+struct IdxCfg {
+  static constexpr int N = 64 * NQ;                  // MMA N: (query, head) pairs
+  static constexpr int ROWB = FP8 ? 128 : 256;       // bytes of one 128-dim vector
+  static constexpr int BOXES = ROWB / 128;           // 128-byte swizzle columns per vector
+  static constexpr int KT_BYTES = 128 * ROWB;        // one 128-key tile
+  static constexpr int Q_BYTES = N * ROWB;           // one query block
+  static constexpr int KSTEPS = ROWB / 32;           // MMAs per tile (K = 32 bytes each)
+  static constexpr int KSTAGES = FP8 ? 8 : (NQ == 1 ? 4 : 2);
+  static constexpr int QSLOTS = 2;
+  static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
+                                   : (2 * N <= 256) ? 256 : 512;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_Q = OFF_K + KSTAGES * KT_BYTES;
+  static constexpr int OFF_W = OFF_Q + QSLOTS * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_W + 2 * N * 4;
+  static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  static constexpr int THREADS = 192;
+  static_assert(N <= 256, "MMA N limit");
+  static_assert(OFF_Q % 1024 == 0 && OFF_W % 1024 == 0, "swizzle atoms need 1 KiB alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Number of 128-key tiles the query block `qb` of sequence b must score: the
+// block's last query sees keys [0, start + t_last].
+template <int NQ>
+__device__ __forceinline__ int seg_len(const int32_t* __restrict__ off, int T, int QB, int seg) {
+  const int b = seg / QB, qb = seg - (seg / QB) * QB;
+  const int E = off[b + 1] - off[b];
+  const int t_last = min(T, (qb + 1) * NQ) - 1;
+  const int L = E - T + t_last + 1;
+  return (L + 127) >> 7;
+}
+
+struct SmemMisc {
+  int seg0, kt0, count, abort, tmem_base, pad[11];
+};
+
+template <int NQ, bool FP8>
+__global__ void __launch_bounds__(192, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const float* __restrict__ w, const float* __restrict__ k_scale,
+                   const int32_t* __restrict__ off, int B, int T, int64_t kv_rows,
+                   float* __restrict__ scores, int64_t ld, int32_t* status) {
+  using C = IdxCfg<NQ, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto k_full = [&](int i) { return bar0 + 8u * i; };
+  auto k_empty = [&](int i) { return bar0 + 8u * (C::KSTAGES + i); };
+  auto q_full = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + i); };
+  auto q_empty = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 2 + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 4 + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 6 + i); };
+  SmemMisc* misc = reinterpret_cast<SmemMisc*>(smem + C::OFF_MISC);
+  volatile int* abort = &misc->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int QB = (T + NQ - 1) / NQ;
+  const int nseg = B * QB;
+
+  // ---- validate offsets and find this CTA's balanced range of work items
+  if (warp == 0) {
+    bool bad = false;
+    for (int b = lane; b < B; b += 32) {
+      const int E = off[b + 1] - off[b];
+      bad |= (off[b] < 0) || (E < T) || ((int64_t)E > ld);
+    }
+    if (lane == 0) bad |= ((int64_t)off[B] > kv_rows);
+    bad = __any_sync(0xffffffffu, bad);
+    int64_t total = 0;
+    if (!bad)
+      for (int base = 0; base < nseg; base += 32) {
+        const int seg = base + lane;
+        int l = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
+        for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        total += l;
+      }
+    const int64_t lo = total * blockIdx.x / gridDim.x;
+    const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+    int seg0 = 0, kt0 = 0;
+    bool found = false;
+    int64_t acc = 0;
+    for (int base = 0; base < nseg && !found && hi > lo; base += 32) {
+      const int seg = base + lane;
+      const int l = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
+      int64_t incl = l;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int64_t excl = incl - l;
+      const bool hit = l > 0 && acc + excl <= lo && lo < acc + incl;
+      const unsigned m = __ballot_sync(0xffffffffu, hit);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        seg0 = __shfl_sync(0xffffffffu, seg, src);
+        kt0 = (int)(lo - acc - __shfl_sync(0xffffffffu, excl, src));
+        found = true;
+      }
+      acc += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      misc->seg0 = seg0;
+      misc->kt0 = kt0;
+      misc->count = (bad || !found) ? 0 : (int)(hi - lo);
+      misc->abort = 0;
+      if (bad && blockIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  const int count = misc->count;
+  if (count == 0) return;
+
+  if (warp == 4 && lane == 0) {
+    for (int i = 0; i < C::KSTAGES; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full(i), 1);
+      mbar_init(q_empty(i), 1 + 4);  // MMA commit + 4 epilogue warps
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + C::OFF_MISC + offsetof(SmemMisc, tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
+
+  // Walk of the CTA's items, identical in every role.
+  int seg = misc->seg0, kt = misc->kt0;
+  int len = seg_len<NQ>(off, T, QB, seg);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer (whole warp)
+    int qord = -1;
+    int issued = 0;
+    for (int item = 0; item < count; ++item) {
+      const int b = seg / QB, qb = seg - b * QB;
+      if (item == 0 || kt == 0) {
+        ++qord;
+        const int qs = qord & 1;
+        bool ok = mbar_wait(q_empty(qs), ((qord >> 1) & 1) ^ 1, abort, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        // per-head weights of this query block, for the epilogue
+        float* wd = w_s + qs * C::N;
+        for (int i = lane; i < C::N; i += 32) {
+          const int t = qb * NQ + i / kHI;
+          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full(qs), C::Q_BYTES);
+          const int y = (b * T + qb * NQ) * kHI;
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_2d(sbase + C::OFF_Q + qs * C::Q_BYTES + bx * (C::N * 128), &tm_q,
+                        bx * (FP8 ? 128 : 64), y, q_full(qs));
+        }
+      }
+      const int st = item % C::KSTAGES;
+      bool ok = mbar_wait(k_empty(st), ((item / C::KSTAGES) & 1) ^ 1, abort, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(k_full(st), C::KT_BYTES);
+        const int y = off[b] + kt * 128;
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_2d(sbase + C::OFF_K + st * C::KT_BYTES + bx * 16384, &tm_k,
+                      bx * (FP8 ? 128 : 64), y, k_full(st));
+      }
+      issued = item + 1;
+      if (++kt == len && item + 1 < count) {
+        ++seg;
+        kt = 0;
+        len = seg_len<NQ>(off, T, QB, seg);
+      }
+    }
+    if (*abort && lane == 0) {  // let copies already in flight land before the CTA exits
+      volatile int never = 0;
+      for (int item = max(0, issued - C::KSTAGES); item < issued; ++item)
+        mbar_wait(k_full(item % C::KSTAGES), (item / C::KSTAGES) & 1, &never, 10000000ull);
+      if (qord >= 0) mbar_wait(q_full(qord & 1), (qord >> 1) & 1, &never, 10000000ull);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = FP8 ? idesc_e4m3(128, C::N) : idesc_bf16(128, C::N);
+      int qord = -1;
+      int issued = 0;
+      for (int item = 0; item < count; ++item) {
+        if (item == 0 || kt == 0) {
+          ++qord;
+          if (!mbar_wait(q_full(qord & 1), (qord >> 1) & 1, abort, kWaitLimitNs)) break;
+        }
+        const int ab = item & 1;
+        if (!mbar_wait(acc_empty(ab), ((item >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+        const int st = item % C::KSTAGES;
+        if (!mbar_wait(k_full(st), (item / C::KSTAGES) & 1, abort, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t a0 = sbase + C::OFF_K + st * C::KT_BYTES;
+        const uint32_t b0 = sbase + C::OFF_Q + (qord & 1) * C::Q_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+          const uint32_t within = (ks & 3) * 32;
+          const uint64_t ad = smem_desc(a0 + (ks >> 2) * 16384 + within, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(b0 + (ks >> 2) * (C::N * 128) + within, 16, 1024, kSwizzle128B);
+          if (FP8)
+            mma_f8_ss(tmem + ab * C::N, ad, bd, idesc, ks > 0);
+          else
+            mma_f16_ss(tmem + ab * C::N, ad, bd, idesc, ks > 0);
+        }
+        tc_commit(k_empty(st));
+        tc_commit(acc_full(ab));
+        issued = item + 1;
+        const bool seg_end = (kt + 1 == len) || (item + 1 == count);
+        if (seg_end) tc_commit(q_empty(qord & 1));
+        if (++kt == len && item + 1 < count) {
+          ++seg;
+          kt = 0;
+          len = seg_len<NQ>(off, T, QB, seg);
+        }
+      }
+      if (*abort && issued > 0) {  // MMAs must finish before TMEM is released
+        volatile int never = 0;
+        const int last = issued - 1;
+        mbar_wait(acc_full(last & 1), (last >> 1) & 1, &never, 10000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    const int row = warp * 32 + lane;  // TMEM lane == key within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    int qord = -1;
+    for (int item = 0; item < count; ++item) {
+      const int b = seg / QB, qb = seg - b * QB;
+      if (item == 0 || kt == 0) {
+        ++qord;  // the producer has staged this block's weights with the query tile
+        bool ok = mbar_wait(q_full(qord & 1), (qord >> 1) & 1, abort, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      const int ab = item & 1;
+      bool ok = mbar_wait(acc_full(ab), (item >> 1) & 1, abort, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int E = off[b + 1] - off[b];
+      const int start = E - T;
+      const int s = kt * 128 + row;
+      float ksc = 1.f;
+      if (FP8 && s < E) ksc = k_scale[off[b] + s];
+#pragma unroll 1
+      for (int q = 0; q < NQ; ++q) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(lane_addr + ab * C::N + q * 64, v0);
+        tmem_ld32(lane_addr + ab * C::N + q * 64 + 32, v1);
+        tc_wait_ld();
+        const float* wq = w_s + (qord & 1) * C::N + q * 64;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          a0 = fmaf(wq[c + 0], fmaxf(__uint_as_float(v0[c + 0]), 0.f), a0);
+          a1 = fmaf(wq[c + 1], fmaxf(__uint_as_float(v0[c + 1]), 0.f), a1);
+          a2 = fmaf(wq[c + 2], fmaxf(__uint_as_float(v0[c + 2]), 0.f), a2);
+          a3 = fmaf(wq[c + 3], fmaxf(__uint_as_float(v0[c + 3]), 0.f), a3);
+        }
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          a0 = fmaf(wq[32 + c + 0], fmaxf(__uint_as_float(v1[c + 0]), 0.f), a0);
+          a1 = fmaf(wq[32 + c + 1], fmaxf(__uint_as_float(v1[c + 1]), 0.f), a1);
+          a2 = fmaf(wq[32 + c + 2], fmaxf(__uint_as_float(v1[c + 2]), 0.f), a2);
+          a3 = fmaf(wq[32 + c + 3], fmaxf(__uint_as_float(v1[c + 3]), 0.f), a3);
+        }
+        const float score = ((a0 + a1) + (a2 + a3)) * ksc;
+        const int t = qb * NQ + q;
+        if (t < T && s < E)
+          scores[((int64_t)b * T + t) * ld + s] = (s <= start + t) ? score : -INFINITY;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(acc_empty(ab));
+        if (kt + 1 == len || item + 1 == count) mbar_arrive(q_empty(qord & 1));  // block done
+      }
+      if (++kt == len && item + 1 < count) {
+        ++seg;
+        kt = 0;
+        len = seg_len<NQ>(off, T, QB, seg);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort) report(status, DSA_ERR_TIMEOUT);
+}
+
+template <int NQ, bool FP8>
+int launch_cfg(const IndexerArgs& a, cudaStream_t stream) {
+  using C = IdxCfg<NQ, FP8>;
+  CUtensorMap tq, tk;
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t box_inner = FP8 ? 128 : 64;
+  const uint64_t q_rows = (uint64_t)a.B * a.T * kHI;
+  if (!make_tmap_2d(&tq, a.q_idx, dt, kDI, q_rows, C::ROWB, box_inner, C::N,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  if (!make_tmap_2d(&tk, a.k_idx, dt, kDI, (uint64_t)a.kv_rows, C::ROWB, box_inner, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  auto kern = indexer_kernel<NQ, FP8>;
+  static bool attr_set = false;  // per template instance
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set = true;
+  }
+  const int grid = device_info().sm_count;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, a.w, a.k_scale, a.offsets, a.B, a.T,
+                                                    a.kv_rows, a.scores, a.ld, a.status);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_indexer(const IndexerArgs& a, cudaStream_t stream) {
+  const bool fp8 = a.idx_dtype == DSA_E4M3;
+  if (a.T == 1) return fp8 ? launch_cfg<1, true>(a, stream) : launch_cfg<1, false>(a, stream);
+  return fp8 ? launch_cfg<4, true>(a, stream) : launch_cfg<4, false>(a, stream);
+}
+
+}  // namespace dsa

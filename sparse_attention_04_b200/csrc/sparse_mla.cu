@@ -1,0 +1,486 @@
+// sparse_mla.cu -- stage 3: absorbed MLA over the selected latent rows.
+//
+// "DeepSeek-V3.2-Exp - Apply sparse mask", MQA decode listing:
+//   scores = (q_nope.kv + q_pe.pe) * softmax_scale,   S~ = S' + M^sel,
+//   p = softmax(S~),   x = p . kv
+// With the cache row stored as one 576-wide vector (512 latent || 64 rope) the
+// two score einsums are one dot product, and only the selected rows carry a
+// finite score, so the kernel gathers exactly those rows and never touches
+// the rest of the cache.
+//
+// Work unit (one CTA, one per SM): query row r, value half v (latent columns
+// [256v, 256v+256)), split sp (a contiguous range of 32-key chunks of the
+// row's index list).  Per chunk i:
+//   S_i = Q . Kv_i^T          M=128 heads, N=32 keys, K=576  (tcgen05, TMEM)
+//   P_i = exp2(S_i*scale*log2e - m)  in bf16                  (CUDA cores)
+//   O  += P_i . Kv_i[:, half] M=128, N=256, K=32              (tcgen05, TMEM)
+// The running max m is only raised when a chunk exceeds it by more than
+// 2^8 (then O and the running sum are rescaled), so P <= 256 and the
+// final O / l is exact softmax.  With more than one split, the unnormalised
+// O and (m, l) go to the workspace and dsa_mla_combine merges them.
+//
+// TMEM: O half in columns [0,256), S in two 32-column buffers at 256 and 288.
+// Shared memory: Q (128 x 576 bf16, 9 swizzled 64-column blocks, by TMA), two
+// stages of 32 gathered rows (cp.async, same swizzled layout), and P.
+// The gathered stage is K-major for Q.K^T and, read as MN-major, the B
+// operand of P.V: one copy of each row serves both products.
+//
+// Roles: warps 0-3 softmax + epilogue (thread = head = TMEM lane),
+//        warps 4-7 row gather, warp 8 TMEM allocator + MMA issuer.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "dsa_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kChunk = 32;
+constexpr int kKB = kDQK / 64;                   // 9 column blocks of 64
+constexpr int kQBytes = kKB * 128 * 128;         // 147456
+constexpr int kKvBytes = kKB * kChunk * 128;     // 36864
+constexpr int kPBytes = 128 * kChunk * 2;        // 8192
+constexpr int kOffQ = 0;
+constexpr int kOffKv = kOffQ + kQBytes;
+constexpr int kOffP = kOffKv + 2 * kKvBytes;
+constexpr int kOffBar = kOffP + kPBytes;
+constexpr int kNumBar = 9;
+constexpr int kOffMisc = kOffBar + kNumBar * 8;
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kThreads = 288;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kIdescQK = idesc_bf16(128, kChunk);
+constexpr uint32_t kIdescPV = idesc_bf16(128, 256, /*b_mn_major=*/true);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffKv % 1024 == 0 && kOffP % 1024 == 0, "alignment");
+
+struct MlaMisc {
+  int tmem_base, abort, n_chunks, last_valid, pad[12];
+};
+
+struct MlaParams {
+  const __nv_bfloat16* kv;
+  const int32_t* off;
+  const int32_t* idx;
+  int T, H, k;
+  int n_splits, cps;  // splits per row, chunks per split
+  float scale_log2;
+  int64_t kv_rows;
+  void* out;
+  int out_bf16;
+  float* lse;
+  float* ws_o;   // [rows][splits][H][512]   (n_splits > 1)
+  float* ws_ml;  // [rows][splits][H][2]
+  int32_t* status;
+};
+
+__device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 && idx < E; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kOffBar;
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto kv_empty = [&](int i) { return bar0 + 8u * (3 + i); };
+  auto s_full = [&](int i) { return bar0 + 8u * (5 + i); };
+  const uint32_t p_full = bar0 + 8u * 7;
+  const uint32_t pv_done = bar0 + 8u * 8;
+  MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
+  volatile int* abort = &misc->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v = blockIdx.x & 1;
+  const int sp = (blockIdx.x >> 1) % p.n_splits;
+  const int r = (blockIdx.x >> 1) / p.n_splits;
+  const int b = r / p.T;
+  const int32_t base_row = p.off[b];
+  const int E = p.off[b + 1] - base_row;
+  const bool geo_ok = base_row >= 0 && E >= p.T && (int64_t)base_row + E <= p.kv_rows;
+  const int32_t* idx_row = p.idx + (int64_t)r * p.k;
+  const int c_begin = sp * p.cps;
+  const int n_chunks_total = (p.k + kChunk - 1) / kChunk;
+  const int c_end = min(c_begin + p.cps, n_chunks_total);
+
+  // ---- how many chunks of this split hold a selected row
+  if (threadIdx.x == 0) {
+    misc->last_valid = -1;
+    misc->abort = 0;
+  }
+  __syncthreads();
+  if (geo_ok) {
+    int lv = -1;
+    for (int j = c_begin * kChunk + threadIdx.x; j < min(c_end * kChunk, p.k); j += kThreads) {
+      const int32_t id = idx_row[j];
+      if (index_ok(id, E)) lv = j;
+      else if (id != -1) report(p.status, DSA_ERR_BAD_INDEX);
+    }
+    if (lv >= 0) atomicMax(&misc->last_valid, lv);
+  } else if (threadIdx.x == 0) {
+    report(p.status, DSA_ERR_BAD_OFFSETS);
+  }
+  __syncthreads();
+  const int n_my = misc->last_valid < 0 ? 0 : misc->last_valid / kChunk - c_begin + 1;
+
+  const int h = threadIdx.x;  // softmax / epilogue threads: head = TMEM lane
+  if (n_my == 0) {
+    // nothing selected in this split: empty partial, or zero output
+    if (warp < 4 && h < p.H) {
+      const int64_t rh = (int64_t)r * p.H + h;
+      if (p.n_splits == 1) {
+        if (p.out_bf16) {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + rh * kDV + 256 * v;
+          for (int c = 0; c < 256; ++c) o[c] = __float2bfloat16(0.f);
+        } else {
+          float* o = reinterpret_cast<float*>(p.out) + rh * kDV + 256 * v;
+          for (int c = 0; c < 256; ++c) o[c] = 0.f;
+        }
+        if (v == 0 && p.lse) p.lse[rh] = -INFINITY;
+      } else {
+        const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
+        float* o = p.ws_o + slot * kDV + 256 * v;
+        for (int c = 0; c < 256; ++c) o[c] = 0.f;
+        if (v == 0) {
+          p.ws_ml[2 * slot] = -INFINITY;
+          p.ws_ml[2 * slot + 1] = 0.f;
+        }
+      }
+    }
+    return;
+  }
+
+  if (warp == 8) {
+    if (lane == 0) {
+      mbar_init(q_full, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(kv_full(i), 128);
+        mbar_init(kv_empty(i), 1);
+        mbar_init(s_full(i), 1);
+      }
+      mbar_init(p_full, 128);
+      mbar_init(pv_done, 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(sbase + kOffMisc + offsetof(MlaMisc, tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
+
+  if (warp == 8) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      for (int kb = 0; kb < kKB; ++kb)
+        tma_load_2d(sbase + kOffQ + kb * 16384, &tm_q, kb * 64, r * p.H, q_full);
+      int done_pv = 0;
+      bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(p_full, j & 1, abort, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t kvb = sbase + kOffKv + (j & 1) * kKvBytes + (4 * v) * (kChunk * 128);
+#pragma unroll
+        for (int ks = 0; ks < kChunk / 16; ++ks) {
+          const uint64_t ad = smem_desc(sbase + kOffP + ks * 256, 128, 512, kSwizzleNone);
+          const uint64_t bd = smem_desc(kvb + ks * 2048, kChunk * 128, 1024, kSwizzle128B);
+          mma_f16_ss(tmem, ad, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc_commit(pv_done);
+        tc_commit(kv_empty(j & 1));
+        done_pv = j + 1;
+        return true;
+      };
+      for (int i = 0; ok && i < n_my; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(kv_full(st), (i >> 1) & 1, abort, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kvb = sbase + kOffKv + st * kKvBytes;
+#pragma unroll 1
+        for (int kb = 0; kb < kKB; ++kb) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = smem_desc(sbase + kOffQ + kb * 16384 + ks * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(kvb + kb * (kChunk * 128) + ks * 32, 16, 1024, kSwizzle128B);
+            mma_f16_ss(tmem + 256 + 32 * st, ad, bd, kIdescQK, (kb | ks) ? 1u : 0u);
+          }
+        }
+        tc_commit(s_full(st));
+        if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(n_my - 1);
+      if (*abort && done_pv > 0) {  // tensor-core work must finish before TMEM is released
+        volatile int never = 0;
+        mbar_wait(pv_done, (done_pv - 1) & 1, &never, 10000000ull);
+      }
+      if (*abort) {
+        volatile int never = 0;
+        mbar_wait(q_full, 0, &never, 10000000ull);
+      }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- row gather
+    const int pt = threadIdx.x - 128;
+    const int jr = pt >> 2, part = pt & 3;
+    const __nv_bfloat16* kv = p.kv;
+    for (int i = 0; i < n_my; ++i) {
+      const int st = i & 1;
+      if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+      const int pos = (c_begin + i) * kChunk + jr;
+      const int32_t id = pos < p.k ? idx_row[pos] : -1;
+      const bool valid = index_ok(id, E);
+      const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
+      const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
+#pragma unroll
+      for (int c = part; c < kDQK / 8; c += 4) {
+        const int kb = c >> 3, cc = c & 7;
+        cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+      }
+      cp_async_commit();
+      // Signal this stage as soon as its rows have landed (the other stage is
+      // meanwhile being consumed by the tensor core).
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(kv_full(st));
+    }
+    cp_async_wait<0>();
+  } else {
+    // -------------------------------------------------------------- softmax + epilogue
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_my; ++i) {
+      const int st = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(st), (i >> 1) & 1, abort, kWaitLimitNs));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[32];
+      tmem_ld32(lane_addr + 256 + 32 * st, sv);
+      tc_wait_ld();
+      float x[32];
+      float mc = -INFINITY;
+      const int pos0 = (c_begin + i) * kChunk;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int32_t id = pos0 + j < p.k ? __ldg(idx_row + pos0 + j) : -1;
+        x[j] = index_ok(id, E) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+        mc = fmaxf(mc, x[j]);
+      }
+      float m_new = m_run;
+      bool resc = false;
+      if (mc > m_run + 8.f) {
+        resc = m_run != -INFINITY;
+        m_new = mc;
+      }
+      const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
+      uint32_t pk[16];
+      float l_chunk = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float p0 = x[j] == -INFINITY ? 0.f : exp2f(x[j] - m_new);
+        const float p1 = x[j + 1] == -INFINITY ? 0.f : exp2f(x[j + 1] - m_new);
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        const float2 back = __bfloat1622float2(pb);
+        l_chunk += back.x + back.y;
+        pk[j / 2] = *reinterpret_cast<const uint32_t*>(&pb);
+      }
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort, kWaitLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+        for (int cb = 0; cb < 8; ++cb) {
+          uint32_t ov[32];
+          tmem_ld32(lane_addr + 32 * cb, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(lane_addr + 32 * cb, ov);
+        }
+        tc_wait_st();
+      }
+      l_run = l_run * alpha + l_chunk;
+      m_run = m_new;
+      // P row h, K-major without swizzle: 8-row x 16-byte core matrices,
+      // 128 bytes apart along K, 512 bytes apart along M.
+      uint8_t* prow = smem + kOffP + (h >> 3) * 512 + (h & 7) * 16;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(prow + c * 128) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_my - 1) & 1, abort, kWaitLimitNs));
+    if (ok) {
+      tc_fence_after();
+      const int64_t rh = (int64_t)r * p.H + h;
+      const bool write = h < p.H;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+      for (int cb = 0; cb < 8; ++cb) {
+        uint32_t ov[32];
+        tmem_ld32(lane_addr + 32 * cb, ov);
+        tc_wait_ld();
+        if (!write) continue;
+        if (p.n_splits == 1) {
+          if (p.out_bf16) {
+            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + rh * kDV + 256 * v + 32 * cb);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                                                 __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
+              }
+              o[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          } else {
+            float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + rh * kDV + 256 * v + 32 * cb);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              o[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv_l, __uint_as_float(ov[4 * q4 + 1]) * inv_l,
+                                  __uint_as_float(ov[4 * q4 + 2]) * inv_l, __uint_as_float(ov[4 * q4 + 3]) * inv_l);
+          }
+        } else {
+          const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
+          float4* o = reinterpret_cast<float4*>(p.ws_o + slot * kDV + 256 * v + 32 * cb);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            o[q4] = make_float4(__uint_as_float(ov[4 * q4]), __uint_as_float(ov[4 * q4 + 1]),
+                                __uint_as_float(ov[4 * q4 + 2]), __uint_as_float(ov[4 * q4 + 3]));
+        }
+      }
+      if (write && v == 0) {
+        if (p.n_splits == 1) {
+          if (p.lse) p.lse[rh] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        } else {
+          const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
+          p.ws_ml[2 * slot] = l_run > 0.f ? m_run : -INFINITY;
+          p.ws_ml[2 * slot + 1] = l_run;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort) report(p.status, DSA_ERR_TIMEOUT);
+}
+
+// Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
+// sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
+__global__ void __launch_bounds__(128)
+    mla_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
+                       int n_splits, void* out, int out_bf16, float* lse) {
+  const int64_t rh = blockIdx.x;  // row * H + head
+  const int64_t r = rh / H, h = rh % H;
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ws_ml[2 * ((r * n_splits + s) * H + h)]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < n_splits; ++s) {
+      const int64_t slot = (r * n_splits + s) * H + h;
+      const float ms = ws_ml[2 * slot];
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L += ws_ml[2 * slot + 1] * f;
+      const float4 o = reinterpret_cast<const float4*>(ws_o + slot * kDV)[threadIdx.x];
+      acc.x += o.x * f;
+      acc.y += o.y * f;
+      acc.z += o.z * f;
+      acc.w += o.w * f;
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (out_bf16) {
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + rh * kDV) + 2 * threadIdx.x;
+    o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  } else {
+    reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + rh * kDV)[threadIdx.x] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+  if (threadIdx.x == 0 && lse) lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace
+
+int mla_num_splits(int n_rows, int k) {
+  const int n_chunks = (k + kChunk - 1) / kChunk;
+  const int sms = device_info().sm_count;
+  int ns = (sms + n_rows - 1) / n_rows;
+  ns = ns < 1 ? 1 : (ns > n_chunks ? n_chunks : ns);
+  const int cps = (n_chunks + ns - 1) / ns;
+  return (n_chunks + cps - 1) / cps;
+}
+
+size_t mla_workspace_bytes(int n_rows, int H, int k) {
+  const int ns = mla_num_splits(n_rows, k);
+  if (ns <= 1) return 0;
+  return (size_t)n_rows * ns * H * (kDV + 2) * sizeof(float);
+}
+
+int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
+  const int n_rows = a.B * a.T;
+  const int ns = mla_num_splits(n_rows, a.k);
+  const int n_chunks = (a.k + kChunk - 1) / kChunk;
+  MlaParams p;
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
+  p.off = a.offsets;
+  p.idx = a.indices;
+  p.T = a.T;
+  p.H = a.H;
+  p.k = a.k;
+  p.n_splits = ns;
+  p.cps = (n_chunks + ns - 1) / ns;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.kv_rows = a.kv_rows;
+  p.out = a.out;
+  p.out_bf16 = a.out_dtype == DSA_BF16;
+  p.lse = a.lse;
+  p.ws_o = nullptr;
+  p.ws_ml = nullptr;
+  p.status = a.status;
+  if (ns > 1) {
+    p.ws_o = reinterpret_cast<float*>(a.workspace);
+    p.ws_ml = p.ws_o + (size_t)n_rows * ns * a.H * kDV;
+  }
+  CUtensorMap tq;
+  if (!make_tmap_2d(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)n_rows * a.H,
+                    kDQK * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set = true;
+  }
+  const int64_t grid = (int64_t)n_rows * ns * 2;
+  sparse_mla_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(tq, p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (ns > 1) {
+    mla_combine_kernel<<<(unsigned)((int64_t)n_rows * a.H), 128, 0, stream>>>(
+        p.ws_o, p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+}  // namespace dsa
