@@ -301,7 +301,7 @@ def run_native(args, rank, world, local):
     # ---- per-stage durations (same kernels, events between stages, in a graph)
     n_prof = min(64, max(8, K))
     ld = step.ld
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_prof)]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(n_prof)]
     ws_mla = step.workspace[_lib.decode_step_workspace_layout(wl.B, max_e, wl.topk, wl.H)[3]:]
     g_prof = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_prof, stream=stream):

@@ -323,6 +323,16 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(acc_empty(ab));
         if (kt + 1 == len || item + 1 == count) mbar_arrive(q_empty(qord & 1));  // block done
       }
+      if (kt + 1 == len && len * 128 < E) {
+        // Keys past the block's causal frontier are never multiplied; they are
+        // masked for every query of the block, so write their -inf here.
+        for (int q = 0; q < NQ; ++q) {
+          const int t = qb * NQ + q;
+          if (t >= T) break;
+          float* srow = scores + ((int64_t)b * T + t) * ld;
+          for (int s2 = len * 128 + threadIdx.x; s2 < E; s2 += 128) srow[s2] = -INFINITY;
+        }
+      }
       if (++kt == len && item + 1 < count) {
         ++seg;
         kt = 0;
