@@ -75,4 +75,23 @@ int mla_num_splits(int n_rows, int k);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
 
+// Launches `kernel` on `stream` with programmatic stream serialisation, so
+// that its prologue overlaps the tail of the previous kernel in the stream.
+// The kernel must call grid_dependency_wait() before reading its inputs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace dsa

@@ -37,7 +37,10 @@ struct IdxCfg {
   static constexpr int KT_BYTES = 128 * ROWB;        // one 128-key tile
   static constexpr int Q_BYTES = N * ROWB;           // one query block
   static constexpr int KSTEPS = ROWB / 32;           // MMAs per tile (K = 32 bytes each)
-  static constexpr int KSTAGES = FP8 ? 8 : (NQ == 1 ? 4 : 2);
+  // Decode (NQ = 1) runs two CTAs per SM with a short ring each, so a 32K-key
+  // row spreads over 2x148 CTAs; prefill keeps one CTA per SM.
+  static constexpr int CTAS_PER_SM = NQ == 1 ? 2 : 1;
+  static constexpr int KSTAGES = NQ == 1 ? (FP8 ? 4 : 2) : (FP8 ? 8 : 2);
   static constexpr int QSLOTS = 2;
   static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
                                    : (2 * N <= 256) ? 256 : 512;
@@ -52,6 +55,7 @@ struct IdxCfg {
   static_assert(N <= 256, "MMA N limit");
   static_assert(OFF_Q % 1024 == 0 && OFF_W % 1024 == 0, "swizzle atoms need 1 KiB alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(CTAS_PER_SM == 1 || SMEM_BYTES * CTAS_PER_SM <= 228 * 1024 - 2048, "two CTAs per SM");
 };
 
 // Number of 128-key tiles the query block `qb` of sequence b must score: the
@@ -70,7 +74,7 @@ struct SmemMisc {
 };
 
 template <int NQ, bool FP8>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
     indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const float* __restrict__ w, const float* __restrict__ k_scale,
                    const int32_t* __restrict__ off, int B, int T, int64_t kv_rows,
@@ -93,6 +97,30 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int QB = (T + NQ - 1) / NQ;
   const int nseg = B * QB;
+
+  // ---- prologue that touches no memory an earlier kernel may still write:
+  // barriers, TMEM, descriptor prefetch.  Overlaps the previous kernel's tail.
+  if (warp == 4 && lane == 0) {
+    for (int i = 0; i < C::KSTAGES; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full(i), 2);       // expect-tx arrival + "weights staged" arrival
+      mbar_init(q_empty(i), 1 + 4);  // MMA commit + 4 epilogue warps
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + C::OFF_MISC + offsetof(SmemMisc, tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  grid_dependency_wait();
+  allow_dependents_launch();
 
   // ---- validate offsets and find this CTA's balanced range of work items
   if (warp == 0) {
@@ -143,37 +171,15 @@ __global__ void __launch_bounds__(192, 1)
       if (bad && blockIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
     }
   }
-  __syncthreads();
-  const int count = misc->count;
-  if (count == 0) return;
-
-  if (warp == 4 && lane == 0) {
-    for (int i = 0; i < C::KSTAGES; ++i) {
-      mbar_init(k_full(i), 1);
-      mbar_init(k_empty(i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full(i), 1);
-      mbar_init(q_empty(i), 1 + 4);  // MMA commit + 4 epilogue warps
-      mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 4);
-    }
-    fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-  }
-  if (warp == 5) {
-    tmem_alloc(sbase + C::OFF_MISC + offsetof(SmemMisc, tmem_base), C::TMEM_COLS);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
+  const int count = misc->count;
 
   // Walk of the CTA's items, identical in every role.
   int seg = misc->seg0, kt = misc->kt0;
-  int len = seg_len<NQ>(off, T, QB, seg);
+  int len = count > 0 ? seg_len<NQ>(off, T, QB, seg) : 0;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer (whole warp)
@@ -186,13 +192,6 @@ __global__ void __launch_bounds__(192, 1)
         const int qs = qord & 1;
         bool ok = mbar_wait(q_empty(qs), ((qord >> 1) & 1) ^ 1, abort, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) break;
-        // per-head weights of this query block, for the epilogue
-        float* wd = w_s + qs * C::N;
-        for (int i = lane; i < C::N; i += 32) {
-          const int t = qb * NQ + i / kHI;
-          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
-        }
-        __syncwarp();
         if (lane == 0) {
           mbar_arrive_expect_tx(q_full(qs), C::Q_BYTES);
           const int y = (b * T + qb * NQ) * kHI;
@@ -200,6 +199,15 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(sbase + C::OFF_Q + qs * C::Q_BYTES + bx * (C::N * 128), &tm_q,
                         bx * (FP8 ? 128 : 64), y, q_full(qs));
         }
+        // per-head weights of this query block, for the epilogue (staged while
+        // the copies fly; the second arrival on q_full publishes them)
+        float* wd = w_s + qs * C::N;
+        for (int i = lane; i < C::N; i += 32) {
+          const int t = qb * NQ + i / kHI;
+          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full(qs));
       }
       const int st = item % C::KSTAGES;
       bool ok = mbar_wait(k_empty(st), ((item / C::KSTAGES) & 1) ^ 1, abort, kWaitLimitNs);
@@ -370,10 +378,11 @@ int launch_cfg(const IndexerArgs& a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
-  const int grid = device_info().sm_count;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, a.w, a.k_scale, a.offsets, a.B, a.T,
-                                                    a.kv_rows, a.scores, a.ld, a.status);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  const int grid = device_info().sm_count * C::CTAS_PER_SM;
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk,
+                                   a.w, a.k_scale, a.offsets, a.B, a.T, a.kv_rows, a.scores, a.ld,
+                                   a.status);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace

@@ -245,6 +245,21 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while its predecessor in the
+// stream is still running; it must call grid_dependency_wait() before it
+// touches memory the predecessor writes (or anything after it reads).  Each
+// kernel calls allow_dependents_launch() once it no longer needs to delay
+// the next kernel's prologue.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t float_order_key(float f) {

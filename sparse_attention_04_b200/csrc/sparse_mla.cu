@@ -106,12 +106,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks_total = (p.k + kChunk - 1) / kChunk;
   const int c_end = min(c_begin + p.cps, n_chunks_total);
 
-  // ---- how many chunks of this split hold a selected row
+  // ---- prologue: barriers, TMEM, and the query tile (q is an input of the
+  // whole step, written before the indexer ran), overlapping the previous
+  // kernel's tail.
   if (threadIdx.x == 0) {
     misc->last_valid = -1;
     misc->abort = 0;
   }
+  if (warp == 8) {
+    if (lane == 0) {
+      mbar_init(q_full, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(kv_full(i), 128);
+        mbar_init(kv_empty(i), 1);
+        mbar_init(s_full(i), 1);
+      }
+      mbar_init(p_full, 128);
+      mbar_init(pv_done, 1);
+      fence_mbar_init();
+      if (geo_ok) {
+        mbar_arrive_expect_tx(q_full, kQBytes);
+        for (int kb = 0; kb < kKB; ++kb)
+          tma_load_2d(sbase + kOffQ + kb * 16384, &tm_q, kb * 64, r * p.H, q_full);
+      }
+    }
+    __syncwarp();
+    tmem_alloc(sbase + kOffMisc + offsetof(MlaMisc, tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
+  grid_dependency_wait();  // the indices come from the previous kernel
+  allow_dependents_launch();
+
+  // ---- how many chunks of this split hold a selected row
   if (geo_ok) {
     int lv = -1;
     for (int j = c_begin * kChunk + threadIdx.x; j < min(c_end * kChunk, p.k); j += kThreads) {
@@ -150,36 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    return;
-  }
-
-  if (warp == 8) {
-    if (lane == 0) {
-      mbar_init(q_full, 1);
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(kv_full(i), 128);
-        mbar_init(kv_empty(i), 1);
-        mbar_init(s_full(i), 1);
-      }
-      mbar_init(p_full, 128);
-      mbar_init(pv_done, 1);
-      fence_mbar_init();
+    if (warp == 8 && lane == 0 && geo_ok) {  // the query tile must land before the CTA exits
+      volatile int never = 0;
+      mbar_wait(q_full, 0, &never, 10000000ull);
     }
-    __syncwarp();
-    tmem_alloc(sbase + kOffMisc + offsetof(MlaMisc, tmem_base), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
-
-  if (warp == 8) {
+  } else if (warp == 8) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kQBytes);
-      for (int kb = 0; kb < kKB; ++kb)
-        tma_load_2d(sbase + kOffQ + kb * 16384, &tm_q, kb * 64, r * p.H, q_full);
       int done_pv = 0;
       bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
       auto issue_pv = [&](int j) -> bool {
@@ -384,27 +391,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
+// Thread c owns columns 4c..4c+3; the split loop is unrolled so its loads are
+// in flight together.
 __global__ void __launch_bounds__(128)
     mla_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
+  __shared__ float s_w[128];
+  __shared__ float s_red[2][4];
+  grid_dependency_wait();  // partials come from the previous kernel
+  allow_dependents_launch();
   const int64_t rh = blockIdx.x;  // row * H + head
   const int64_t r = rh / H, h = rh % H;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ws_ml[2 * ((r * n_splits + s) * H + h)]);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float m = -INFINITY, l = 0.f;
+  if ((int)threadIdx.x < n_splits) {
+    const int64_t slot = (r * n_splits + threadIdx.x) * H + h;
+    m = ws_ml[2 * slot];
+    l = ws_ml[2 * slot + 1];
+  }
+  float M = m;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_red[0][warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
+  const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+  s_w[threadIdx.x] = f;
+  float L = l * f;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if (lane == 0) s_red[1][warp] = L;
+  __syncthreads();
+  L = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = 0.f;
   if (M != -INFINITY) {
+    const float4* base = reinterpret_cast<const float4*>(ws_o + (r * n_splits * H + h) * kDV) + threadIdx.x;
+    const int64_t stride4 = (int64_t)H * kDV / 4;  // between consecutive splits
+#pragma unroll 8
     for (int s = 0; s < n_splits; ++s) {
-      const int64_t slot = (r * n_splits + s) * H + h;
-      const float ms = ws_ml[2 * slot];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += ws_ml[2 * slot + 1] * f;
-      const float4 o = reinterpret_cast<const float4*>(ws_o + slot * kDV)[threadIdx.x];
-      acc.x += o.x * f;
-      acc.y += o.y * f;
-      acc.z += o.z * f;
-      acc.w += o.w * f;
+      const float4 o = __ldg(base + s * stride4);
+      const float fs = s_w[s];
+      acc.x = fmaf(o.x, fs, acc.x);
+      acc.y = fmaf(o.y, fs, acc.y);
+      acc.z = fmaf(o.z, fs, acc.z);
+      acc.w = fmaf(o.w, fs, acc.w);
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -421,11 +451,21 @@ __global__ void __launch_bounds__(128)
 
 }  // namespace
 
+#ifndef DSA_MLA_MIN_CHUNKS_PER_SPLIT
+#define DSA_MLA_MIN_CHUNKS_PER_SPLIT 2
+#endif
+
+// Splits of a row's index list: enough CTAs (two per split, one per value
+// half) to cover the SMs when there are few rows, but at least
+// DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split, since every split costs one
+// query-tile load and one 128 x 512 fp32 partial.
 int mla_num_splits(int n_rows, int k) {
   const int n_chunks = (k + kChunk - 1) / kChunk;
   const int sms = device_info().sm_count;
+  int max_splits = n_chunks / DSA_MLA_MIN_CHUNKS_PER_SPLIT;
+  if (max_splits < 1) max_splits = 1;
   int ns = (sms + n_rows - 1) / n_rows;
-  ns = ns < 1 ? 1 : (ns > n_chunks ? n_chunks : ns);
+  ns = ns < 1 ? 1 : (ns > max_splits ? max_splits : ns);
   const int cps = (n_chunks + ns - 1) / ns;
   return (n_chunks + cps - 1) / cps;
 }
@@ -473,12 +513,14 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   const int64_t grid = (int64_t)n_rows * ns * 2;
-  sparse_mla_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(tq, p);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, p) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   if (ns > 1) {
-    mla_combine_kernel<<<(unsigned)((int64_t)n_rows * a.H), 128, 0, stream>>>(
-        p.ws_o, p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(128), 0, stream,
+                   (const float*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
   }
   return DSA_OK;
 }

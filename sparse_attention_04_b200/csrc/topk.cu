@@ -7,15 +7,25 @@
 // equals +0.0, so the result is unique and deterministic.
 //
 // One CTA (1024 threads) per query row.  The valid positions of a row are the
-// causal prefix s < L = min(end_pos, start + t + 1).  Algorithm:
-//   1. map every score to an order-preserving 32-bit key (larger = better);
-//   2. radix-select the k-th largest key tau with three digit passes
-//      (11, 11, 10 bits, most significant first) over shared-memory
-//      histograms, narrowing to the elements that share the digits found;
-//   3. one stable compaction pass in position order keeps every key > tau and
-//      the first (k - #greater) keys == tau, writing positions ascending.
-// Keys stay in shared memory when the row fits (<= kSmemKeys), else each pass
-// re-reads the scores (they were just written and sit in L2).
+// causal prefix s < L = end_pos - T + t + 1.  Scores are mapped to
+// order-preserving 32-bit keys (larger score = larger key).
+//
+// Main path (L <= 131072):
+//   A. histogram of the top 12 key bits (shared atomics);
+//      a suffix scan finds the bin d* holding the k-th largest key;
+//   B. one pass marks, in a bitmap whose word w covers positions 32w..32w+31
+//      (thread-owned, so no atomics), every key whose bin is above d*, and
+//      copies the keys of bin d* (the candidates) into shared memory;
+//   C. two digit passes over the candidates only fix the exact k-th key tau
+//      and how many keys equal to tau are kept (the lowest positions, found by
+//      a scan over a second bitmap);
+//   D. one block scan of the words' popcounts writes the kept positions in
+//      ascending order.
+// Fallback (more candidates than the buffer holds, e.g. massive ties, or
+// very long rows): three 11/11/10-bit digit passes over the whole row and a
+// stable scan-based compaction.
+#include <cooperative_groups.h>
+
 #include "dsa_internal.h"
 #include "sm100.cuh"
 
@@ -24,21 +34,30 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
-constexpr int kSmemKeys = 48 * 1024;  // 192 KiB of keys
+constexpr int kBins12 = 4096;            // top-12-bit histogram
+constexpr int kMaxWords = 4096;          // bitmap words: rows up to 131072 positions
+constexpr int kWordsPerThread = kMaxWords / kThreads;
+constexpr int kCap = 8192;               // candidate buffer (keys of the threshold bin)
+constexpr int kFallbackSmemKeys = 2 * kMaxWords + 2 * kCap;  // the same bytes reused as keys
 
 struct TopkSmem {
-  uint32_t hist[kBins];
   uint32_t warp_tot[kWarps];
+  uint32_t carry;
   uint32_t sel_digit;
   uint32_t sel_remaining;
-  uint32_t carry;
-  uint32_t pad;
+  uint32_t n_cand;
+  uint32_t pad[12];
+  uint32_t hist[kBins12];
 };
+// dynamic layout after TopkSmem: bitmap[kMaxWords] | eqmap[kMaxWords] |
+// cand_key[kCap] | cand_pos[kCap]   (the fallback reuses it as a key array)
+constexpr size_t kSmemBytes = sizeof(TopkSmem) + sizeof(uint32_t) * (2 * kMaxWords + 2 * kCap);
 
-// Exclusive block-wide scan of one uint32 per thread; returns the thread's
-// exclusive prefix and writes the block total to *total.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, TopkSmem& sm, uint32_t* total) {
+// Exclusive block-wide scan of one uint32 per thread (NT threads); returns the
+// thread's exclusive prefix and writes the block total to *total.
+template <int NT = kThreads, class SM>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, SM& sm, uint32_t* total) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -49,15 +68,15 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, TopkSmem& sm, ui
   if (lane == 31) sm.warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t t = sm.warp_tot[lane];
+    const uint32_t t = lane < NW ? sm.warp_tot[lane] : 0u;
     uint32_t ti = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t u = __shfl_up_sync(0xffffffffu, ti, o);
       if (lane >= o) ti += u;
     }
-    sm.warp_tot[lane] = ti - t;  // exclusive warp offsets
-    if (lane == 31) sm.carry = ti;
+    if (lane < NW) sm.warp_tot[lane] = ti - t;  // exclusive warp offsets
+    if (lane == NW - 1) sm.carry = ti;
   }
   __syncthreads();
   const uint32_t res = sm.warp_tot[warp] + incl - v;
@@ -66,101 +85,131 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, TopkSmem& sm, ui
   return res;
 }
 
-__device__ __forceinline__ uint32_t load_key(const float* __restrict__ row, const uint32_t* keys,
-                                             bool in_smem, int s) {
-  return in_smem ? keys[s] : float_order_key(__ldg(row + s));
+// Finds, over `nb` histogram bins in descending digit order, the bin holding
+// the `remaining`-th largest element.  Writes sm.sel_digit and sm.sel_remaining
+// (the rank inside that bin).  Every thread must call it.
+template <int NT = kThreads, class SM>
+__device__ __forceinline__ void select_bin(SM& sm, const uint32_t* hist, int nb, uint32_t remaining) {
+  const int per = nb / NT;  // bins per thread, descending (at most 16)
+  uint32_t c[16];
+  uint32_t sum = 0;
+  const int top = nb - 1 - per * (int)threadIdx.x;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    c[j] = j < per ? hist[top - j] : 0u;
+    sum += c[j];
+  }
+  uint32_t tot;
+  uint32_t above = block_excl_scan<NT>(sum, sm, &tot);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < per && above < remaining && remaining <= above + c[j]) {
+      sm.sel_digit = (uint32_t)(top - j);
+      sm.sel_remaining = remaining - above;
+    }
+    above += c[j];
+  }
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off,
-                int B, int T, int k, int32_t* __restrict__ indices, int32_t* status) {
-  extern __shared__ uint8_t smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem));
+__device__ __forceinline__ uint32_t load_key(const float* __restrict__ row, int s) {
+  return float_order_key(__ldg(row + s));
+}
 
-  const int r = blockIdx.x;
-  const int b = r / T, t = r - (r / T) * T;
-  int32_t* out = indices + (int64_t)r * k;
-  const int E = off[b + 1] - off[b];
-  if (E < T || (int64_t)E > ld || off[b] < 0) {
-    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = -1;
-    if (threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
-    return;
+// Keys of positions 32w .. 32w+31; bits of *valid_bits mark positions < L.
+__device__ __forceinline__ void load_word(const float* __restrict__ row, int L, int w, uint32_t (&kk)[32],
+                                          uint32_t* valid_bits) {
+  const int s0 = 32 * w;
+  if (s0 + 32 <= L) {
+    const float4* p = reinterpret_cast<const float4*>(row + s0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = __ldg(p + j);
+      kk[4 * j + 0] = float_order_key(v.x);
+      kk[4 * j + 1] = float_order_key(v.y);
+      kk[4 * j + 2] = float_order_key(v.z);
+      kk[4 * j + 3] = float_order_key(v.w);
+    }
+    *valid_bits = 0xffffffffu;
+  } else {
+    uint32_t vb = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const bool ok = s0 + j < L;
+      kk[j] = ok ? load_key(row, s0 + j) : 0u;
+      vb |= (ok ? 1u : 0u) << j;
+    }
+    *valid_bits = vb;
   }
-  const int L = E - T + t + 1;  // causal prefix: every valid position
-  const float* row = scores + (int64_t)r * ld;
+}
 
-  if (L <= k) {  // every valid position is kept
-    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < L ? j : -1;
-    return;
+// Writes the positions of the set bits of bitmap[0 .. n_words) ascending into out.
+template <class SM>
+__device__ __forceinline__ void emit_bitmap(SM& sm, const uint32_t* bitmap, int n_words, int32_t* out) {
+  const int w0 = threadIdx.x * kWordsPerThread;
+  uint32_t cnt = 0;
+  for (int j = 0; j < kWordsPerThread; ++j)
+    if (w0 + j < n_words) cnt += __popc(bitmap[w0 + j]);
+  uint32_t tot;
+  uint32_t pos = block_excl_scan(cnt, sm, &tot);
+  for (int j = 0; j < kWordsPerThread; ++j) {
+    if (w0 + j >= n_words) break;
+    uint32_t bits = bitmap[w0 + j];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      out[pos++] = 32 * (w0 + j) + b;
+    }
   }
+}
 
-  const bool in_smem = L <= kSmemKeys;
-  // ---- digit passes
+// Three 11/11/10-bit digit passes over the whole row and a stable compaction.
+template <int NT = kThreads, class SM>
+__device__ void radix_select_fallback(SM& sm, uint32_t* keys, int key_cap, const float* __restrict__ row, int L,
+                                      int k, int32_t* __restrict__ out) {
+  const bool in_smem = L <= key_cap;
   uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
+  uint32_t* hist = sm.hist;
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const uint32_t nb = 1u << widths[pass];
-    for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    for (int i = threadIdx.x; i < kBins12; i += NT) hist[i] = 0;
     __syncthreads();
-    if (pass == 0 && in_smem) {
-      for (int s = threadIdx.x; s < L; s += kThreads) {
-        const uint32_t key = float_order_key(__ldg(row + s));
-        keys[s] = key;
-        atomicAdd(&sm.hist[key >> shift], 1u);
+    for (int s = threadIdx.x; s < L; s += NT) {
+      uint32_t key;
+      if (pass == 0) {
+        key = load_key(row, s);
+        if (in_smem) keys[s] = key;
+      } else {
+        key = in_smem ? keys[s] : load_key(row, s);
       }
-    } else {
-      for (int s = threadIdx.x; s < L; s += kThreads) {
-        const uint32_t key = load_key(row, keys, in_smem, s);
-        if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1u);
-      }
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
-    // Bins in descending digit order: thread i owns digits nb-1-2i and nb-2-2i
-    // (nb/2 <= 1024 threads cover them all).
-    const int d_hi = (int)nb - 1 - 2 * (int)threadIdx.x;
-    const uint32_t c_hi = d_hi >= 0 ? sm.hist[d_hi] : 0u;
-    const uint32_t c_lo = d_hi - 1 >= 0 ? sm.hist[d_hi - 1] : 0u;
-    uint32_t tot;
-    const uint32_t above = block_excl_scan(c_hi + c_lo, sm, &tot);
-    if (d_hi >= 0) {
-      if (above < remaining && remaining <= above + c_hi) {
-        sm.sel_digit = (uint32_t)d_hi;
-        sm.sel_remaining = remaining - above;
-      } else if (d_hi - 1 >= 0 && above + c_hi < remaining && remaining <= above + c_hi + c_lo) {
-        sm.sel_digit = (uint32_t)(d_hi - 1);
-        sm.sel_remaining = remaining - above - c_hi;
-      }
-    }
-    __syncthreads();
+    select_bin<NT>(sm, hist, nb, remaining);
     prefix |= sm.sel_digit << shift;
-    pmask |= (nb - 1) << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
     remaining = sm.sel_remaining;
     __syncthreads();
   }
-  const uint32_t tau = prefix;
-  const uint32_t need_eq = remaining;  // keys equal to tau to keep, lowest positions first
-
-  // ---- stable compaction in position order
-  constexpr int V = 8;  // positions per thread per tile
+  const uint32_t tau = prefix, need_eq = remaining;
+  constexpr int V = 8;
   uint32_t gt_carry = 0, eq_carry = 0;
 #pragma unroll 1
-  for (int base = 0; base < L; base += kThreads * V) {
+  for (int base = 0; base < L; base += NT * V) {
     const int s0 = base + threadIdx.x * V;
     uint32_t kk[V];
     uint32_t gt = 0, eq = 0;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int s = s0 + j;
-      kk[j] = s < L ? load_key(row, keys, in_smem, s) : 0u;
+      kk[j] = s < L ? (in_smem ? keys[s] : load_key(row, s)) : 0u;
       gt += (s < L && kk[j] > tau);
       eq += (s < L && kk[j] == tau);
     }
     uint32_t tot;
-    const uint32_t packed = block_excl_scan(gt | (eq << 16), sm, &tot);
+    const uint32_t packed = block_excl_scan<NT>(gt | (eq << 16), sm, &tot);
     uint32_t g = gt_carry + (packed & 0xFFFFu);
     uint32_t q = eq_carry + (packed >> 16);
 #pragma unroll
@@ -178,25 +227,531 @@ __global__ void __launch_bounds__(kThreads, 1)
     gt_carry += tot & 0xFFFFu;
     eq_carry += tot >> 16;
   }
-  for (int j = threadIdx.x; j < k; j += kThreads)
-    if (j >= k) out[j] = -1;  // k_eff == k whenever L > k: nothing to pad
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off,
+                int B, int T, int k, int32_t* __restrict__ indices, int32_t* status) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem));
+  uint32_t* eqmap = bitmap + kMaxWords;
+  uint32_t* cand_key = eqmap + kMaxWords;
+  uint32_t* cand_pos = cand_key + kCap;
+
+  grid_dependency_wait();  // scores come from the previous kernel
+  allow_dependents_launch();
+  const int r = blockIdx.x;
+  const int b = r / T, t = r - (r / T) * T;
+  int32_t* out = indices + (int64_t)r * k;
+  const int E = off[b + 1] - off[b];
+  if (E < T || (int64_t)E > ld || off[b] < 0) {
+    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = -1;
+    if (threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
+    return;
+  }
+  const int L = E - T + t + 1;  // causal prefix: every valid position
+  const float* row = scores + (int64_t)r * ld;
+
+  if (L <= k) {  // every valid position is kept
+    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < L ? j : -1;
+    return;
+  }
+  if (L > kMaxWords * 32) {
+    radix_select_fallback(sm, bitmap, kFallbackSmemKeys, row, L, k, out);
+    return;
+  }
+
+  const int n_words = (L + 31) >> 5;
+  for (int i = threadIdx.x; i < kBins12; i += kThreads) sm.hist[i] = 0;
+  if (threadIdx.x == 0) sm.n_cand = 0;
+  __syncthreads();
+
+  // ---- A: histogram of the top 12 bits
+  auto hist_word = [&](const uint32_t (&kk)[32], uint32_t vb) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if ((vb >> j) & 1u) atomicAdd(&sm.hist[kk[j] >> 20], 1u);
+  };
+#pragma unroll 1
+  for (int i = 0; i < kWordsPerThread; ++i) {
+    const int w = threadIdx.x + i * kThreads;
+    if (w >= n_words) break;
+    uint32_t kk[32], vb = 0;
+    load_word(row, L, w, kk, &vb);
+    hist_word(kk, vb);
+  }
+  __syncthreads();
+  select_bin(sm, sm.hist, kBins12, (uint32_t)k);
+  const uint32_t dstar = sm.sel_digit;
+  const uint32_t need_in_bin = sm.sel_remaining;  // how many keys of bin d* are kept
+
+  // ---- B: bitmap of keys above bin d*, candidates of bin d*
+#pragma unroll 1
+  for (int i = 0; i < kWordsPerThread; ++i) {
+    const int w = threadIdx.x + i * kThreads;
+    if (w >= n_words) break;
+    uint32_t kk[32], vb;
+    load_word(row, L, w, kk, &vb);  // second read of the row: it is in L2
+    uint32_t bits = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t bin = kk[j] >> 20;
+      if ((vb >> j) & 1u) {
+        if (bin > dstar) {
+          bits |= 1u << j;
+        } else if (bin == dstar) {
+          const uint32_t slot = atomicAdd(&sm.n_cand, 1u);
+          if (slot < kCap) {
+            cand_key[slot] = kk[j];
+            cand_pos[slot] = 32 * w + j;
+          }
+        }
+      }
+    }
+    bitmap[w] = bits;
+    eqmap[w] = 0;
+  }
+  __syncthreads();
+  const uint32_t n_cand = sm.n_cand;
+  if (n_cand > kCap) {  // too many keys share the threshold bin: exact slow path
+    radix_select_fallback(sm, bitmap, kFallbackSmemKeys, row, L, k, out);
+    return;
+  }
+
+  // ---- C: exact threshold among the candidates (low 20 bits: 10 + 10)
+  uint32_t prefix = dstar << 20, pmask = 0xFFF00000u, remaining = need_in_bin;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    for (int i = threadIdx.x; i < 1024; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (uint32_t c = threadIdx.x; c < n_cand; c += kThreads) {
+      const uint32_t key = cand_key[c];
+      if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
+    }
+    __syncthreads();
+    select_bin(sm, sm.hist, 1024, remaining);
+    prefix |= sm.sel_digit << shift;
+    pmask |= 1023u << shift;
+    remaining = sm.sel_remaining;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix, need_eq = remaining;
+  for (uint32_t c = threadIdx.x; c < n_cand; c += kThreads) {
+    const uint32_t key = cand_key[c], s = cand_pos[c];
+    if (key > tau) atomicOr(&bitmap[s >> 5], 1u << (s & 31));
+    else if (key == tau) atomicOr(&eqmap[s >> 5], 1u << (s & 31));
+  }
+  __syncthreads();
+  // keep the need_eq lowest positions whose key equals tau
+  {
+    const int w0 = threadIdx.x * kWordsPerThread;
+    uint32_t cnt = 0;
+    for (int j = 0; j < kWordsPerThread; ++j)
+      if (w0 + j < n_words) cnt += __popc(eqmap[w0 + j]);
+    uint32_t tot;
+    uint32_t rank = block_excl_scan(cnt, sm, &tot);
+    for (int j = 0; j < kWordsPerThread; ++j) {
+      if (w0 + j >= n_words) break;
+      uint32_t bits = eqmap[w0 + j], keep = 0;
+      while (bits && rank < need_eq) {
+        const uint32_t low = bits & (0u - bits);
+        keep |= low;
+        bits ^= low;
+        ++rank;
+      }
+      if (keep) bitmap[w0 + j] |= keep;
+    }
+  }
+  __syncthreads();
+  // ---- D: ascending output (exactly k positions: L > k here)
+  emit_bitmap(sm, bitmap, n_words, out);
+}
+
+
+// ============================================================================
+// Cluster variant for long rows: CS CTAs (one thread-block cluster) per row,
+// each owning a contiguous, word-aligned slice of positions.  The CTAs
+// exchange data by writing into each other's shared memory (remote stores,
+// absorbed by the next cluster barrier) in four rounds:
+//   1  every CTA sends each bin range of its 12-bit histogram to the range's
+//      owner (CTA c owns bins [c*4096/CS, (c+1)*4096/CS))
+//   2  every owner sums its range and sends it, with its total, to all CTAs;
+//      each CTA then finds bin d* (the k-th largest key's bin) locally
+//   3  every CTA marks its keys above d* in its bitmap (one warp per 32
+//      positions, via ballots) and sends its candidates (keys in bin d*) and
+//      counts to rank 0
+//   4  rank 0 fixes the exact threshold tau over all candidates and sends
+//      each CTA tau, its tie quota and its output offset
+// after which every CTA writes its kept positions independently.
+template <int CS>
+struct ClusterCfg {
+  static constexpr int kSliceMax = 131072 / CS;          // positions per CTA
+  static constexpr int kSliceWords = kSliceMax / 32;
+  static constexpr int kPart = kBins12 / CS;               // bins owned per CTA
+  static constexpr int kLocalCap = 2048;                   // candidates kept per CTA
+  static constexpr int kPerSrc = 8192 / CS;                // candidates each CTA may send rank 0
+  static constexpr int kThreads = 256;
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kWordsPerThread = kSliceWords / kThreads;
+};
+
+template <int CS>
+struct ClusterSmem {
+  using C = ClusterCfg<CS>;
+  uint32_t warp_tot[32];
+  uint32_t carry, sel_digit, sel_remaining, n_cand;
+  uint32_t above_count, pad0[3];
+  uint32_t tau, need_eq, eq_base, out_base, mode, pad1[3];
+  uint32_t all_tot[CS];                // every owner's bin-range total
+  uint32_t g_cnt[CS], g_above[CS];     // rank 0: candidates and above-counts per CTA
+  uint32_t cnt_gt[CS], cnt_eq[CS];     // rank 0 scratch
+  uint32_t hist[kBins12];              // local histogram, later scratch
+  uint32_t recv_hist[CS][C::kPart];    // owner: the range from every CTA
+  uint32_t all_part[kBins12];          // every CTA: the summed histogram
+  uint32_t bitmap[C::kSliceWords];
+  uint32_t eqmap[C::kSliceWords];
+  uint32_t cand_key[C::kLocalCap];
+  uint32_t cand_pos[C::kLocalCap];
+  uint32_t keys[C::kSliceMax];
+  uint32_t g_key[CS][C::kPerSrc];      // rank 0: candidates from every CTA
+};
+
+template <int CS>
+__global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
+    topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B,
+                        int T, int k, int32_t* __restrict__ indices, int32_t* status) {
+  using Cfg = ClusterCfg<CS>;
+  constexpr int kThreads = Cfg::kThreads, kWarps = Cfg::kWarps;
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  ClusterSmem<CS>& sm = *reinterpret_cast<ClusterSmem<CS>*>(smem_raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  grid_dependency_wait();  // scores come from the previous kernel
+  allow_dependents_launch();
+  const int r = blockIdx.x / CS;
+  const int b = r / T, t = r - (r / T) * T;
+  int32_t* out = indices + (int64_t)r * k;
+  const int E = off[b + 1] - off[b];
+  if (E < T || (int64_t)E > ld || off[b] < 0) {  // same verdict in every CTA of the cluster
+    if (rank == 0) {
+      for (int j = threadIdx.x; j < k; j += kThreads) out[j] = -1;
+      if (threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
+    }
+    return;
+  }
+  const int L = E - T + t + 1;
+  const float* row = scores + (int64_t)r * ld;
+  if (L <= k) {
+    if (rank == 0)
+      for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < L ? j : -1;
+    return;
+  }
+  // slice of this CTA, word aligned (the host sends only rows of <= 131072 positions here)
+  const int S = (((L + CS - 1) / CS) + 31) & ~31;
+  const int s_lo = min(rank * S, L), s_hi = min(s_lo + S, L);
+  const int n = s_hi - s_lo;
+  const int n_words = (n + 31) >> 5;
+
+  // ---- round 1: keys of the slice, local histogram, ranges to their owners
+  for (int i = threadIdx.x; i < kBins12; i += kThreads) sm.hist[i] = 0;
+  if (threadIdx.x == 0) {
+    sm.n_cand = 0;
+    sm.above_count = 0;
+  }
+  __syncthreads();
+  {
+    const float4* r4 = reinterpret_cast<const float4*>(row + s_lo);  // s_lo is a multiple of 32
+    uint4* k4 = reinterpret_cast<uint4*>(sm.keys);
+    const int n4 = n >> 2;
+    for (int i4 = threadIdx.x; i4 < n4; i4 += kThreads) {
+      const float4 v = __ldg(r4 + i4);
+      const uint4 kk = make_uint4(float_order_key(v.x), float_order_key(v.y), float_order_key(v.z),
+                                  float_order_key(v.w));
+      k4[i4] = kk;
+      atomicAdd(&sm.hist[kk.x >> 20], 1u);
+      atomicAdd(&sm.hist[kk.y >> 20], 1u);
+      atomicAdd(&sm.hist[kk.z >> 20], 1u);
+      atomicAdd(&sm.hist[kk.w >> 20], 1u);
+    }
+    for (int s = 4 * n4 + threadIdx.x; s < n; s += kThreads) {
+      const uint32_t key = float_order_key(__ldg(row + s_lo + s));
+      sm.keys[s] = key;
+      atomicAdd(&sm.hist[key >> 20], 1u);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins12; i += kThreads) {
+    const int q = i / Cfg::kPart;
+    cluster.map_shared_rank(&sm.recv_hist[0][0], q)[rank * Cfg::kPart + (i - q * Cfg::kPart)] = sm.hist[i];
+  }
+  cluster.sync();  // 1
+
+  // ---- round 2: owners sum their range and send it to everyone
+  {
+    uint32_t mine = 0;
+    for (int i = threadIdx.x; i < Cfg::kPart; i += kThreads) {
+      uint32_t sum = 0;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) sum += sm.recv_hist[q][i];
+      mine += sum;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) cluster.map_shared_rank(sm.all_part, q)[rank * Cfg::kPart + i] = sum;
+    }
+    uint32_t tot;
+    block_excl_scan<kThreads>(mine, sm, &tot);
+    if (threadIdx.x < CS) cluster.map_shared_rank(sm.all_tot, (int)threadIdx.x)[rank] = tot;
+  }
+  cluster.sync();  // 2
+
+  // bin d* holding the k-th largest key: all data is local now
+  uint32_t dstar, need_in_bin;
+  {
+    __shared__ uint32_t s_owner, s_above;
+    if (threadIdx.x == 0) {  // owners in descending bin order: rank CS-1 holds the highest bins
+      uint32_t above = 0;
+      int owner = 0;
+      for (int q = CS - 1; q >= 0; --q) {
+        if (above + sm.all_tot[q] >= (uint32_t)k) {
+          owner = q;
+          break;
+        }
+        above += sm.all_tot[q];
+      }
+      s_owner = (uint32_t)owner;
+      s_above = above;
+    }
+    __syncthreads();
+    const int owner = (int)s_owner;
+    for (int i = threadIdx.x; i < 1024; i += kThreads)
+      sm.hist[i] = i < Cfg::kPart ? sm.all_part[owner * Cfg::kPart + i] : 0u;
+    __syncthreads();
+    select_bin<kThreads>(sm, sm.hist, 1024, (uint32_t)k - s_above);
+    dstar = (uint32_t)(owner * Cfg::kPart) + sm.sel_digit;
+    need_in_bin = sm.sel_remaining;
+  }
+
+  // ---- round 3: bitmap of keys above d*, candidates in d*, counts to rank 0
+  {
+    uint32_t above_local = 0;
+    for (int w = warp; w < Cfg::kSliceWords; w += kWarps) {
+      const int s = 32 * w + lane;
+      const bool valid = w < n_words && s < n;
+      const uint32_t key = valid ? sm.keys[s] : 0u;
+      const uint32_t bin = key >> 20;
+      const uint32_t up = __ballot_sync(0xffffffffu, valid && bin > dstar);
+      const uint32_t cand = __ballot_sync(0xffffffffu, valid && bin == dstar);
+      if (cand) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sm.n_cand, (uint32_t)__popc(cand));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (valid && bin == dstar) {
+          const uint32_t slot = base + __popc(cand & ((1u << lane) - 1u));
+          if (slot < (uint32_t)Cfg::kLocalCap) {
+            sm.cand_key[slot] = key;
+            sm.cand_pos[slot] = (uint32_t)s;
+          }
+        }
+      }
+      if (lane == 0) {
+        sm.bitmap[w] = up;
+        sm.eqmap[w] = 0;
+      }
+      above_local += __popc(up);
+    }
+    if (lane == 0 && above_local) atomicAdd(&sm.above_count, above_local);
+    __syncthreads();
+    const uint32_t nc = sm.n_cand;
+    ClusterSmem<CS>* r0 = cluster.map_shared_rank(&sm, 0);
+    const bool fits = nc <= (uint32_t)Cfg::kPerSrc;
+    if (fits)
+      for (uint32_t c = threadIdx.x; c < nc; c += kThreads) r0->g_key[rank][c] = sm.cand_key[c];
+    if (threadIdx.x == 0) {
+      r0->g_cnt[rank] = fits ? nc : 0xFFFFFFFFu;  // overflow marker
+      r0->g_above[rank] = sm.above_count;
+    }
+  }
+  cluster.sync();  // 3
+
+  // ---- round 4: rank 0 fixes the exact threshold and every CTA's offsets
+  if (rank == 0) {
+    __shared__ uint32_t s_goff[CS + 1], s_mode;
+    if (threadIdx.x == 0) {
+      uint32_t total = 0, bad = 0;
+      for (int q = 0; q < CS; ++q) {
+        bad |= sm.g_cnt[q] == 0xFFFFFFFFu;
+        s_goff[q] = total;
+        total += bad ? 0u : sm.g_cnt[q];
+      }
+      s_goff[CS] = total;
+      s_mode = bad ? 1u : 0u;
+    }
+    if (threadIdx.x < CS) sm.cnt_gt[threadIdx.x] = sm.cnt_eq[threadIdx.x] = 0;
+    __syncthreads();
+    if (s_mode == 0) {
+      uint32_t prefix = dstar << 20, pmask = 0xFFF00000u, remaining = need_in_bin;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0;
+        for (int i = threadIdx.x; i < 1024; i += kThreads) sm.hist[i] = 0;
+        __syncthreads();
+        for (int q = 0; q < CS; ++q)
+          for (uint32_t c = threadIdx.x; c < sm.g_cnt[q]; c += kThreads) {
+            const uint32_t key = sm.g_key[q][c];
+            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
+          }
+        __syncthreads();
+        select_bin<kThreads>(sm, sm.hist, 1024, remaining);
+        prefix |= sm.sel_digit << shift;
+        pmask |= 1023u << shift;
+        remaining = sm.sel_remaining;
+        __syncthreads();
+      }
+      const uint32_t tau = prefix, need_eq = remaining;
+      for (int q = 0; q < CS; ++q)
+        for (uint32_t c = threadIdx.x; c < sm.g_cnt[q]; c += kThreads) {
+          const uint32_t key = sm.g_key[q][c];
+          if (key > tau) atomicAdd(&sm.cnt_gt[q], 1u);
+          else if (key == tau) atomicAdd(&sm.cnt_eq[q], 1u);
+        }
+      __syncthreads();
+      if (threadIdx.x < CS) {
+        const int q = (int)threadIdx.x;
+        uint32_t eq_base = 0, out_base = 0;
+        for (int p = 0; p < q; ++p) {
+          const uint32_t taken = eq_base >= need_eq ? 0u : min(sm.cnt_eq[p], need_eq - eq_base);
+          eq_base += sm.cnt_eq[p];
+          out_base += sm.g_above[p] + sm.cnt_gt[p] + taken;
+        }
+        ClusterSmem<CS>* dst = cluster.map_shared_rank(&sm, q);
+        dst->tau = tau;
+        dst->need_eq = need_eq;
+        dst->eq_base = eq_base;
+        dst->out_base = out_base;
+        dst->mode = 0;
+      }
+    } else if (threadIdx.x < CS) {
+      cluster.map_shared_rank(&sm, (int)threadIdx.x)->mode = 1;
+    }
+  }
+  cluster.sync();  // 4: no remote shared-memory access after this point
+
+  if (sm.mode == 1) {  // a CTA had too many keys in bin d*: rank 0 redoes the row alone
+    if (rank == 0) radix_select_fallback<kThreads>(sm, sm.keys, Cfg::kSliceMax, row, L, k, out);
+    return;
+  }
+  const uint32_t tau = sm.tau, need_eq = sm.need_eq;
+  const uint32_t n_cand = min(sm.n_cand, (uint32_t)Cfg::kLocalCap);
+  for (uint32_t c = threadIdx.x; c < n_cand; c += kThreads) {
+    const uint32_t key = sm.cand_key[c], s = sm.cand_pos[c];
+    if (key > tau) atomicOr(&sm.bitmap[s >> 5], 1u << (s & 31));
+    else if (key == tau) atomicOr(&sm.eqmap[s >> 5], 1u << (s & 31));
+  }
+  __syncthreads();
+  {  // keys equal to tau: keep those whose rank over the whole row is below need_eq
+    const int w0 = threadIdx.x * Cfg::kWordsPerThread;
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int j = 0; j < Cfg::kWordsPerThread; ++j) cnt += __popc(sm.eqmap[w0 + j]);
+    uint32_t tot;
+    uint32_t rk = sm.eq_base + block_excl_scan<kThreads>(cnt, sm, &tot);
+#pragma unroll
+    for (int j = 0; j < Cfg::kWordsPerThread; ++j) {
+      uint32_t bits = sm.eqmap[w0 + j], keep = 0;
+      while (bits && rk < need_eq) {
+        const uint32_t low = bits & (0u - bits);
+        keep |= low;
+        bits ^= low;
+        ++rk;
+      }
+      if (keep) sm.bitmap[w0 + j] |= keep;
+    }
+  }
+  __syncthreads();
+  {  // ascending output of this slice at its offset
+    const int w0 = threadIdx.x * Cfg::kWordsPerThread;
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int j = 0; j < Cfg::kWordsPerThread; ++j) cnt += __popc(sm.bitmap[w0 + j]);
+    uint32_t tot;
+    uint32_t pos = sm.out_base + block_excl_scan<kThreads>(cnt, sm, &tot);
+#pragma unroll
+    for (int j = 0; j < Cfg::kWordsPerThread; ++j) {
+      uint32_t bits = sm.bitmap[w0 + j];
+      while (bits) {
+        const int bb = __ffs(bits) - 1;
+        bits &= bits - 1;
+        out[pos++] = s_lo + 32 * (w0 + j) + bb;
+      }
+    }
+  }
+}
+
+template <int CS>
+int launch_cluster(const TopkArgs& a, cudaStream_t stream) {
+  auto kern = topk_cluster_kernel<CS>;
+  const size_t smem = sizeof(ClusterSmem<CS>);
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (CS > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.B * a.T * CS));
+  cfg.blockDim = dim3(ClusterCfg<CS>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices,
+                                           a.status);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
 
+// Rows longer than kClusterMinLd positions go to the cluster kernel (16 CTAs
+// per row when there are few rows, else 8); shorter rows (prefill) take one
+// CTA each.
+#ifndef DSA_TOPK_CLUSTER_MIN_LD
+#define DSA_TOPK_CLUSTER_MIN_LD 8192
+#endif
+
+#ifndef DSA_TOPK_FEW_ROWS_CLUSTER
+#define DSA_TOPK_FEW_ROWS_CLUSTER 16
+#endif
+
 int launch_topk(const TopkArgs& a, cudaStream_t stream) {
-  const size_t smem = sizeof(TopkSmem) + sizeof(uint32_t) * kSmemKeys;
+  const int rows = a.B * a.T;
+  if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072) {
+    if (DSA_TOPK_FEW_ROWS_CLUSTER == 16 && rows * 16 <= 2 * device_info().sm_count)
+      return launch_cluster<16>(a, stream);
+    return launch_cluster<8>(a, stream);
+  }
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
     attr_set = true;
   }
-  const int rows = a.B * a.T;
-  topk_kernel<<<rows, kThreads, smem, stream>>>(a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices,
-                                               a.status);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  const cudaError_t e = launch_pdl(topk_kernel, dim3(rows), dim3(kThreads), kSmemBytes, stream, a.scores,
+                                   a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace dsa

@@ -1,0 +1,62 @@
+"""dsa_topk on constructed score rows, bit-exact against the oracle's selection
+(larger score first, then lower position; -0.0 == +0.0; ascending output, -1
+padding).  Covers both the bitmap path and its fallback (threshold bin with
+more candidates than the buffer, rows longer than the bitmap)."""
+import pytest
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(rows, k, T=1):
+    """rows: list of 1-D float32 CPU tensors, one per sequence (T=1 decode rows)."""
+    from sparse_attention_04_b200 import _lib
+    dev = torch.device("cuda:0")
+    eps = [r.numel() for r in rows]
+    ld = (max(eps) + 3) // 4 * 4
+    sc = torch.full((len(rows), ld), float("nan"), dtype=torch.float32)
+    for i, r in enumerate(rows):
+        sc[i, :r.numel()] = r
+    off = torch.tensor([0] + list(torch.tensor(eps).cumsum(0).tolist()), dtype=torch.int32)
+    out = torch.empty((len(rows), k), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _lib.topk(sc.to(dev), ld, off.to(dev), len(rows), T, k, out, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    want = oracle.topk(sc.double(), off, len(rows), T, k)
+    return out.cpu(), want
+
+
+def _gen(n, seed):
+    return torch.randn(n, generator=torch.Generator().manual_seed(seed))
+
+
+@pytest.mark.parametrize("n,k", [(32768, 2048), (32768 + 7, 2048), (131072, 2048), (131072 + 5, 2048),
+                                 (5000, 4), (2049, 2048), (70000, 1)])
+def test_random_rows(cuda_device, n, k):
+    got, want = _run([_gen(n, n)], k)
+    assert torch.equal(got, want)
+
+
+def test_massive_ties_take_the_fallback(cuda_device):
+    got, want = _run([torch.full((40000,), 0.5), torch.zeros(9000)], 2048)
+    assert torch.equal(got, want)
+    assert got[0].tolist() == list(range(2048))
+
+
+def test_signed_zeros_and_few_distinct_values(cuda_device):
+    g = torch.Generator().manual_seed(3)
+    alphabet = torch.tensor([-0.0, 0.0, 1.0, -1.0, 2.5, 1e-30, -1e-30, float("-inf")])
+    rows = [alphabet[torch.randint(0, 8, (30000,), generator=g)],
+            torch.randn(30000, generator=g).round(decimals=1),     # ~60 distinct values, heavy ties
+            torch.randn(12345, generator=g) * 1e-20]
+    got, want = _run(rows, 2048)
+    assert torch.equal(got, want)
+
+
+def test_batch_of_ragged_rows(cuda_device):
+    rows = [_gen(n, 100 + n) for n in (1, 31, 32, 33, 2047, 2048, 2049, 4096, 50000)]
+    got, want = _run(rows, 2048)
+    assert torch.equal(got, want)
