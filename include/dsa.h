@@ -132,6 +132,35 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
                     int32_t* dev_status, void* stream);
 
 /*
+ * Stage 3 without a caller workspace.  The paper has no counterpart: this is
+ * a convenience of this library, not a step of the method.
+ *
+ * For callers that cannot allocate device memory where they issue the step
+ * (a plugin inside a runtime that owns all device memory and offers no
+ * allocator, a serving loop whose memory is fixed at start-up, code that may
+ * not call cudaMalloc on that path).  Same arguments, layouts and results as
+ * dsa_sparse_mla, minus the workspace: the split partials live in a scratch
+ * array of DSA_NOALLOC_SCRATCH_BYTES (64 MiB) built into the library, which
+ * every GPU that loads the library holds until the process exits.
+ *   - A call that needs more scratch than that (dsa_sparse_mla_workspace_size
+ *     above the limit; e.g. 128..147 rows at H = 128, k = 2048) returns
+ *     DSA_ERR_WORKSPACE before launching anything.
+ *   - The first call on each device looks the scratch address up with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.  It allocates nothing, ever.
+ *   - All calls on a device share the one scratch array: calls that may run
+ *     concurrently on the GPU (different streams, no ordering between them)
+ *     race and corrupt each other's results.  Order them on one stream.
+ *   - Nothing in the scratch needs to start at zero: every value a call reads
+ *     was written earlier in the same call.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int dsa_sparse_mla_noalloc(const void* q, const void* kv, const int32_t* offsets,
+                           const int32_t* indices, int B, int T, int H, int k, float scale,
+                           int64_t kv_rows, void* out, int out_dtype, float* lse,
+                           int32_t* dev_status, void* stream);
+
+/*
  * Where, inside a decode-step workspace, the step leaves its intermediates
  * (byte offsets; the scores pitch is returned in *ld_scores).  For tests and
  * tools that want to look at stage outputs; the layout may change between

@@ -22,7 +22,7 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
-           "dsa_decode_step", "dsa_decode_step_workspace_layout")
+           "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc")
 
 
 class DSAError(RuntimeError):
@@ -46,6 +46,7 @@ def _load():
         "dsa_decode_step_workspace_size": ([I, I, I, I], SZ),
         "dsa_decode_step": ([P, P, P, P, I, P, P, P, I, I, I64, I, I, F, P, I, P, P, SZ, P, P], I),
         "dsa_decode_step_workspace_layout": ([I, I, I, I, P, P, P, P], I),
+        "dsa_sparse_mla_noalloc": ([P, P, P, P, I, I, I, I, F, I64, P, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -115,6 +116,15 @@ def sparse_mla(q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out, lse=Non
                               _p(out), out_code, _p(lse), _p(workspace), ws_bytes, _p(status),
                               _stream(stream)),
            "dsa_sparse_mla")
+
+
+def sparse_mla_noalloc(q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out, lse=None, status=None,
+                       stream=None):
+    """dsa_sparse_mla_noalloc: dsa_sparse_mla with the library's built-in scratch (no workspace)."""
+    out_code = DSA_BF16 if out.dtype == torch.bfloat16 else DSA_F32
+    _check(lib.dsa_sparse_mla_noalloc(_p(q), _p(kv), _p(offsets), _p(indices), B, T, H, k, float(scale), kv_rows,
+                                      _p(out), out_code, _p(lse), _p(status), _stream(stream)),
+           "dsa_sparse_mla_noalloc")
 
 
 def decode_step_workspace_size(B, max_end_pos, k, H) -> int:
