@@ -226,7 +226,8 @@ def run_native(args, rank, world, local):
                                 device_id=dev)
     wl = I.WORKLOADS[args.workload]
     if wl.T != 1:
-        raise SystemExit("bench times decode workloads (T = 1)")
+        run_prefill_only(args, rank, world, dev)
+        return
     base = I.make_inputs(wl, dev)
     E = base.end_pos
     max_e = max(E)
@@ -340,6 +341,8 @@ def run_native(args, rank, world, local):
 
     # ---- end to end: host buffers in, host result out, through the C ABI
     e2e = run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world)
+    del copies
+    prefill = None if args.no_prefill else run_prefill(dev, stream, peaks)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
@@ -351,6 +354,8 @@ def run_native(args, rank, world, local):
                        "l2": f"cold: {n_copies} rotating cache copies (> 3x L2)",
                        "algorithmic_bytes_per_step": sb["step"]},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * K, "clocks": clk}
+    if prefill is not None:
+        line["prefill_indexer"] = prefill
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = base.to("cpu")
         v, cores, text = time_oracle(wl, cpu, n_steps=3, seconds_per_step_budget=args.cpu_seconds / 3)
@@ -419,6 +424,114 @@ def run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world):
             "note": "caches stay resident; per step the new token's q_I, w, q, key row and latent row go in, the output comes out"}
 
 
+def prefill_indexer_flops(T, E):
+    """Useful indexer flops of one causal prefill: 2*64*128 per (query, visible key)."""
+    return 2 * 64 * 128 * sum(min(E, E - T + t + 1) for t in range(T))
+
+
+def run_prefill(dev, stream, peaks, reps=20):
+    """Causal 4K prefill (B=1, T=4096): the indexer against the bf16 tensor
+    peak, and the whole staged path (indexer, top-k, sparse MLA) for context.
+
+    Three copies of the inputs and of the score matrix rotate between
+    launches (about 400 MB in all, above 3x L2).  Events on the launching
+    stream bracket a CUDA graph of `reps` launches."""
+    import torch
+    from sparse_attention_04_b200 import _lib
+    from sparse_attention_04_b200 import inputs as I
+    wl = I.WORKLOADS["prefill4k"]
+    B, T, H, k = wl.B, wl.T, wl.H, wl.topk
+    E = wl.end_pos
+    n_copies = 3
+    copies = [I.make_inputs(wl, dev)]
+    for _ in range(n_copies - 1):
+        c = copies[0]
+        copies.append(I.Inputs(wl, c.end_pos, c.offsets, c.q_idx.clone(), c.w.clone(), c.k_idx.clone(), None,
+                               c.q, c.kv))
+    ld = (E + 3) // 4 * 4
+    scores = [torch.empty((B * T, ld), dtype=torch.float32, device=dev) for _ in range(n_copies)]
+    indices = torch.empty((B * T, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(16, _lib.sparse_mla_workspace_size(B, T, H, k)), dtype=torch.uint8, device=dev)
+
+    def indexer(i):
+        x = copies[i % n_copies]
+        _lib.indexer_scores(x.q_idx, x.w, x.k_idx, None, x.offsets, B, T, x.rows, scores[i % n_copies], ld,
+                            status=status)
+
+    def staged(i):
+        x = copies[i % n_copies]
+        indexer(i)
+        _lib.topk(scores[i % n_copies], ld, x.offsets, B, T, k, indices, status=status)
+        _lib.sparse_mla(x.q, x.kv, x.offsets, indices, B, T, H, k, wl.scale, x.rows, out, lse=lse, workspace=ws,
+                        status=status)
+
+    def timed(fn, n):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            g.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3 / n
+
+    t_idx = timed(indexer, reps)
+    t_all = timed(staged, max(2, reps // 4))
+    if int(status.item()) != 0:
+        raise SystemExit("prefill: device status " + _lib.status_string(int(status.item())))
+    flops = prefill_indexer_flops(T, E)
+    try:
+        peak, src = float(peaks["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    achieved = flops / t_idx / 1e12
+    return {"workload": "prefill4k", "kernel": "indexer", "bound": "tensor", "us": round(t_idx * 1e6, 2),
+            "flops": flops, "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_source": src,
+            "staged_step_us": round(t_all * 1e6, 1),
+            "note": "causal lower triangle only; 3 rotating input and score copies"}
+
+
+def run_prefill_only(args, rank, world, dev):
+    """`--workload prefill4k`: the causal prefill indexer alone, as its own JSON line."""
+    import torch
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        peaks = {}
+    stream = torch.cuda.Stream(dev)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    res = run_prefill(dev, stream, peaks, reps=max(1, args.steps))
+    clk = clocks.stop()
+    t_max = reduce_max(res["us"] * 1e-6, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        line = {"metric": "DSA causal prefill indexer TFLOP/s (T=4096, lower triangle)",
+                "value": round(res["flops"] * world / t_max / 1e12, 1), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": 3, "ms_per_step": round(t_max * 1e3, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1) bf16)", "config": {"workload": "prefill4k", "B": 1, "T": 4096,
+                                                                     "end_pos": 4096, "heads": 64},
+                "roofline": {k: res[k] for k in ("bound", "achieved", "peak", "unit", "frac", "peak_source")},
+                "prefill_indexer": res, "clocks": clk}
+        print(json.dumps(line), flush=True)
+
+
 def load_traffic(workload, kernel):
     """DRAM bytes per launch from the committed ncu summary for this kernel and
     workload, if one exists for the current kernel version; else None."""
@@ -472,12 +585,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "batched", "fp8", "tiny"])
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "batched", "fp8", "tiny", "prefill4k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--graph-steps", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the causal 4K prefill indexer measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -11,15 +11,21 @@
 // so every epilogue thread owns one key (one TMEM lane) and forms
 // sum_h w * max(0, D) from its own registers -- no cross-lane reduction.
 //
-// Roles (one CTA per SM, persistent over a balanced range of a flat list of
+// Roles (persistent CTAs, each over a balanced range of a flat list of
 // (sequence, query block, key tile) items):
-//   warps 0-3  epilogue: TMEM -> registers, ReLU, weight, head sum, mask, store
-//   warp  4    TMA producer: key tiles into a ring of stages, query blocks
-//              into two slots (reloaded only when the query block changes)
-//   warp  5    TMEM allocator + MMA issuer (one thread)
+//   epilogue warps  TMEM -> registers, ReLU, weight, head sum, mask, store
+//                   (4 warps for decode; 8 for prefill, two per TMEM lane
+//                   quarter, each taking half of the block's queries)
+//   producer warp   TMA: key tiles into a ring of stages, query blocks into
+//                   two slots (reloaded only when the query block changes);
+//                   between loads it writes -inf past each prefill row's
+//                   causal frontier, where no tile is multiplied
+//   MMA warp        TMEM allocator + MMA issuer (one thread)
 // Key tiles and query blocks land in shared memory in the 128-byte-swizzled
 // K-major layout the MMA descriptors describe; accumulators are double
 // buffered in TMEM so the epilogue of tile i overlaps the MMA of tile i+1.
+// The work split charges every query block one extra unit on top of its
+// tiles (prefill), for its query reload and pipeline restart.
 #include <cuda.h>
 
 #include "dsa_internal.h"
@@ -42,6 +48,11 @@ struct IdxCfg {
   static constexpr int CTAS_PER_SM = NQ == 1 ? 2 : 1;
   static constexpr int KSTAGES = NQ == 1 ? (FP8 ? 4 : 2) : (FP8 ? 8 : 2);
   static constexpr int QSLOTS = 2;
+  static constexpr int EPI_WARPS = NQ == 1 ? 4 : 8;
+  static constexpr int QPW = NQ * 4 / EPI_WARPS;     // queries per epilogue warp
+  static constexpr int SEG_COST = NQ == 1 ? 0 : 1;   // balance units per query block
+  static constexpr int PRODUCER = EPI_WARPS;         // warp indices of the two roles
+  static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
                                    : (2 * N <= 256) ? 256 : 512;
   static constexpr int OFF_K = 0;
@@ -51,7 +62,8 @@ struct IdxCfg {
   static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 32 * (EPI_WARPS + 2);
+  static_assert(NQ % (EPI_WARPS / 4) == 0, "queries split evenly over the warps of a lane quarter");
   static_assert(N <= 256, "MMA N limit");
   static_assert(OFF_Q % 1024 == 0 && OFF_W % 1024 == 0, "swizzle atoms need 1 KiB alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -70,11 +82,31 @@ __device__ __forceinline__ int seg_len(const int32_t* __restrict__ off, int T, i
 }
 
 struct SmemMisc {
-  int seg0, kt0, count, abort, tmem_base, pad[11];
+  int seg0, kt0, count, abort, tmem_base, bad, pad[10];
 };
 
+// 64-head weighted ReLU sum of one key for one query: sum_h w[h]*max(0, d[h]),
+// d[0..31] in v0 and d[32..63] in v1, on packed two-lane fp32 FMAs.
+__device__ __forceinline__ float head_sum64(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
+                                            const float* __restrict__ wq) {
+  float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                 make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 64; c += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(wq + c);
+    const uint32_t* v = c < 32 ? v0 : v1;
+    const int cc = c & 31;
+    const float2 x01 = make_float2(fmaxf(__uint_as_float(v[cc + 0]), 0.f), fmaxf(__uint_as_float(v[cc + 1]), 0.f));
+    const float2 x23 = make_float2(fmaxf(__uint_as_float(v[cc + 2]), 0.f), fmaxf(__uint_as_float(v[cc + 3]), 0.f));
+    const int j = (c >> 2) & 1;
+    a[2 * j] = __ffma2_rn(x01, make_float2(w4.x, w4.y), a[2 * j]);
+    a[2 * j + 1] = __ffma2_rn(x23, make_float2(w4.z, w4.w), a[2 * j + 1]);
+  }
+  return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+}
+
 template <int NQ, bool FP8>
-__global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
+__global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTAS_PER_SM)
     indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const float* __restrict__ w, const float* __restrict__ k_scale,
                    const int32_t* __restrict__ off, int B, int T, int64_t kv_rows,
@@ -100,29 +132,32 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
 
   // ---- prologue that touches no memory an earlier kernel may still write:
   // barriers, TMEM, descriptor prefetch.  Overlaps the previous kernel's tail.
-  if (warp == 4 && lane == 0) {
+  if (warp == C::PRODUCER && lane == 0) {
     for (int i = 0; i < C::KSTAGES; ++i) {
       mbar_init(k_full(i), 1);
       mbar_init(k_empty(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full(i), 2);       // expect-tx arrival + "weights staged" arrival
-      mbar_init(q_empty(i), 1 + 4);  // MMA commit + 4 epilogue warps
+      mbar_init(q_full(i), 2);                  // expect-tx arrival + "weights staged" arrival
+      mbar_init(q_empty(i), 1 + C::EPI_WARPS);  // MMA commit + every epilogue warp
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 4);
+      mbar_init(acc_empty(i), C::EPI_WARPS);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
   }
-  if (warp == 5) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(sbase + C::OFF_MISC + offsetof(SmemMisc, tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
   grid_dependency_wait();
   allow_dependents_launch();
 
-  // ---- validate offsets and find this CTA's balanced range of work items
+  // ---- validate offsets and find this CTA's balanced range of work units.
+  // Segment (query block) s costs SEG_COST + len_s units; its tiles are the
+  // last len_s of them.  The CTA takes units [lo, hi) and scores the tiles
+  // among them, which are contiguous in the flat tile list.
   if (warp == 0) {
     bool bad = false;
     for (int b = lane; b < B; b += 32) {
@@ -135,39 +170,45 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
     if (!bad)
       for (int base = 0; base < nseg; base += 32) {
         const int seg = base + lane;
-        int l = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
-        for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        total += l;
+        int64_t u = seg < nseg ? seg_len<NQ>(off, T, QB, seg) + C::SEG_COST : 0;
+        for (int o = 16; o; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        total += u;
       }
     const int64_t lo = total * blockIdx.x / gridDim.x;
     const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
     int seg0 = 0, kt0 = 0;
+    int64_t count = 0;
     bool found = false;
     int64_t acc = 0;
-    for (int base = 0; base < nseg && !found && hi > lo; base += 32) {
+    for (int base = 0; base < nseg && acc < hi && !bad; base += 32) {
       const int seg = base + lane;
-      const int l = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
-      int64_t incl = l;
+      const int len = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
+      const int64_t u = seg < nseg ? len + C::SEG_COST : 0;
+      int64_t incl = u;
       for (int o = 1; o < 32; o <<= 1) {
         const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      const int64_t excl = incl - l;
-      const bool hit = l > 0 && acc + excl <= lo && lo < acc + incl;
-      const unsigned m = __ballot_sync(0xffffffffu, hit);
-      if (m) {
+      const int64_t tile_lo = acc + incl - len, tile_hi = acc + incl;  // this segment's tile units
+      const int64_t ov_lo = max(tile_lo, lo), ov_hi = min(tile_hi, hi);
+      int64_t ov = ov_hi > ov_lo ? ov_hi - ov_lo : 0;
+      const unsigned m = __ballot_sync(0xffffffffu, ov > 0);
+      if (!found && m) {
         const int src = __ffs(m) - 1;
         seg0 = __shfl_sync(0xffffffffu, seg, src);
-        kt0 = (int)(lo - acc - __shfl_sync(0xffffffffu, excl, src));
+        kt0 = (int)__shfl_sync(0xffffffffu, ov_lo - tile_lo, src);
         found = true;
       }
+      for (int o = 16; o; o >>= 1) ov += __shfl_xor_sync(0xffffffffu, ov, o);
+      count += ov;
       acc += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) {
       misc->seg0 = seg0;
       misc->kt0 = kt0;
-      misc->count = (bad || !found) ? 0 : (int)(hi - lo);
+      misc->count = (bad || !found) ? 0 : (int)count;
       misc->abort = 0;
+      misc->bad = bad ? 1 : 0;
       if (bad && blockIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
     }
   }
@@ -181,8 +222,38 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
   int seg = misc->seg0, kt = misc->kt0;
   int len = count > 0 ? seg_len<NQ>(off, T, QB, seg) : 0;
 
-  if (warp == 4) {
+  if (warp == C::PRODUCER) {
     // ------------------------------------------------------------ producer (whole warp)
+    // -inf past the causal frontier of the rows r = blockIdx.x (mod gridDim.x):
+    // keys beyond the last tile of a row's query block are never multiplied.
+    // Written 512 bytes per step, a few steps after each load (decode rows
+    // have nothing to fill).
+    const int64_t n_rows = (int64_t)B * T;
+    int64_t f_r = (T > 1 && !misc->bad) ? (int64_t)blockIdx.x : n_rows;
+    int64_t f_pos = 0, f_end = 0;
+    float* f_row = scores;
+    auto fill = [&](int steps) {
+      while (steps > 0) {
+        if (f_pos >= f_end) {
+          if (f_r >= n_rows) return;
+          const int fb = (int)(f_r / T), ft = (int)(f_r - (int64_t)fb * T);
+          f_pos = (int64_t)seg_len<NQ>(off, T, QB, fb * QB + ft / NQ) * 128;
+          f_end = off[fb + 1] - off[fb];
+          f_row = scores + f_r * ld;
+          f_r += gridDim.x;
+          continue;
+        }
+        const int64_t s0 = f_pos + 4 * lane;  // f_pos is a multiple of 128: 16-byte aligned
+        if (s0 + 4 <= f_end) {
+          *reinterpret_cast<float4*>(f_row + s0) = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        } else {
+          for (int j = 0; j < 4; ++j)
+            if (s0 + j < f_end) f_row[s0 + j] = -INFINITY;
+        }
+        f_pos += 128;
+        --steps;
+      }
+    };
     int qord = -1;
     int issued = 0;
     for (int item = 0; item < count; ++item) {
@@ -220,19 +291,21 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
                       bx * (FP8 ? 128 : 64), y, k_full(st));
       }
       issued = item + 1;
+      fill(4);
       if (++kt == len && item + 1 < count) {
         ++seg;
         kt = 0;
         len = seg_len<NQ>(off, T, QB, seg);
       }
     }
+    if (!*abort) fill(1 << 30);
     if (*abort && lane == 0) {  // let copies already in flight land before the CTA exits
       volatile int never = 0;
       for (int item = max(0, issued - C::KSTAGES); item < issued; ++item)
         mbar_wait(k_full(item % C::KSTAGES), (item / C::KSTAGES) & 1, &never, 10000000ull);
       if (qord >= 0) mbar_wait(q_full(qord & 1), (qord >> 1) & 1, &never, 10000000ull);
     }
-  } else if (warp == 5) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = FP8 ? idesc_e4m3(128, C::N) : idesc_bf16(128, C::N);
@@ -278,10 +351,14 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 0-3)
-    const int row = warp * 32 + lane;  // TMEM lane == key within the tile
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------------------ epilogue warps
+    const int qd = warp & 3;                    // TMEM lane quarter of this warp
+    const int q_lo = (warp >> 2) * C::QPW;      // its share of the block's queries
+    const int row = qd * 32 + lane;             // TMEM lane == key within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     int qord = -1;
+    int cur_b = -1, E = 0, start = 0;
+    int32_t base_row = 0;
     for (int item = 0; item < count; ++item) {
       const int b = seg / QB, qb = seg - b * QB;
       if (item == 0 || kt == 0) {
@@ -289,38 +366,27 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
         bool ok = mbar_wait(q_full(qord & 1), (qord >> 1) & 1, abort, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
+      if (b != cur_b) {
+        cur_b = b;
+        base_row = off[b];
+        E = off[b + 1] - base_row;
+        start = E - T;
+      }
       const int ab = item & 1;
       bool ok = mbar_wait(acc_full(ab), (item >> 1) & 1, abort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int E = off[b + 1] - off[b];
-      const int start = E - T;
       const int s = kt * 128 + row;
       float ksc = 1.f;
-      if (FP8 && s < E) ksc = k_scale[off[b] + s];
+      if (FP8 && s < E) ksc = k_scale[base_row + s];
 #pragma unroll 1
-      for (int q = 0; q < NQ; ++q) {
+      for (int qq = 0; qq < C::QPW; ++qq) {
+        const int q = q_lo + qq;
         uint32_t v0[32], v1[32];
         tmem_ld32(lane_addr + ab * C::N + q * 64, v0);
         tmem_ld32(lane_addr + ab * C::N + q * 64 + 32, v1);
         tc_wait_ld();
-        const float* wq = w_s + (qord & 1) * C::N + q * 64;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          a0 = fmaf(wq[c + 0], fmaxf(__uint_as_float(v0[c + 0]), 0.f), a0);
-          a1 = fmaf(wq[c + 1], fmaxf(__uint_as_float(v0[c + 1]), 0.f), a1);
-          a2 = fmaf(wq[c + 2], fmaxf(__uint_as_float(v0[c + 2]), 0.f), a2);
-          a3 = fmaf(wq[c + 3], fmaxf(__uint_as_float(v0[c + 3]), 0.f), a3);
-        }
-#pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          a0 = fmaf(wq[32 + c + 0], fmaxf(__uint_as_float(v1[c + 0]), 0.f), a0);
-          a1 = fmaf(wq[32 + c + 1], fmaxf(__uint_as_float(v1[c + 1]), 0.f), a1);
-          a2 = fmaf(wq[32 + c + 2], fmaxf(__uint_as_float(v1[c + 2]), 0.f), a2);
-          a3 = fmaf(wq[32 + c + 3], fmaxf(__uint_as_float(v1[c + 3]), 0.f), a3);
-        }
-        const float score = ((a0 + a1) + (a2 + a3)) * ksc;
+        const float score = head_sum64(v0, v1, w_s + (qord & 1) * C::N + q * 64) * ksc;
         const int t = qb * NQ + q;
         if (t < T && s < E)
           scores[((int64_t)b * T + t) * ld + s] = (s <= start + t) ? score : -INFINITY;
@@ -331,16 +397,6 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
         mbar_arrive(acc_empty(ab));
         if (kt + 1 == len || item + 1 == count) mbar_arrive(q_empty(qord & 1));  // block done
       }
-      if (kt + 1 == len && len * 128 < E) {
-        // Keys past the block's causal frontier are never multiplied; they are
-        // masked for every query of the block, so write their -inf here.
-        for (int q = 0; q < NQ; ++q) {
-          const int t = qb * NQ + q;
-          if (t >= T) break;
-          float* srow = scores + ((int64_t)b * T + t) * ld;
-          for (int s2 = len * 128 + threadIdx.x; s2 < E; s2 += 128) srow[s2] = -INFINITY;
-        }
-      }
       if (++kt == len && item + 1 < count) {
         ++seg;
         kt = 0;
@@ -350,7 +406,7 @@ __global__ void __launch_bounds__(192, IdxCfg<NQ, FP8>::CTAS_PER_SM)
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

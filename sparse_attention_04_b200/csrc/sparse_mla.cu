@@ -48,6 +48,8 @@ constexpr int kOffP = kOffKv + 2 * kKvBytes;
 constexpr int kOffBar = kOffP + kPBytes;
 constexpr int kNumBar = 9;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
+constexpr int kStageRow = 1040;                  // epilogue staging: 1 KiB + 16 per head
+static_assert(128 * kStageRow <= kQBytes, "the staged output fits where the query tile was");
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mbar_init(q_full, 1);
       for (int i = 0; i < 2; ++i) {
-        mbar_init(kv_full(i), 128);
+        mbar_init(kv_full(i), 64);  // the gather group of that stage
         mbar_init(kv_empty(i), 1);
         mbar_init(s_full(i), 1);
       }
@@ -233,10 +235,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- row gather
+    // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
+    // the two groups run independently, so both stages are in flight from
+    // the start and a group waits only for its own copies before it signals.
     const int pt = threadIdx.x - 128;
-    const int jr = pt >> 2, part = pt & 3;
+    const int grp = pt >> 6, gt = pt & 63;
+    const int jr = gt >> 1, part = gt & 1;
     const __nv_bfloat16* kv = p.kv;
-    for (int i = 0; i < n_my; ++i) {
+    for (int i = grp; i < n_my; i += 2) {
       const int st = i & 1;
       if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
       const int pos = (c_begin + i) * kChunk + jr;
@@ -244,14 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = index_ok(id, E);
       const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
       const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
-#pragma unroll
-      for (int c = part; c < kDQK / 8; c += 4) {
+#pragma unroll 4
+      for (int c = part; c < kDQK / 8; c += 2) {
         const int kb = c >> 3, cc = c & 7;
         cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
       }
       cp_async_commit();
-      // Signal this stage as soon as its rows have landed (the other stage is
-      // meanwhile being consumed by the tensor core).
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(kv_full(st));
@@ -328,48 +332,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_my - 1) & 1, abort, kWaitLimitNs));
     if (ok) {
+      // Every MMA has completed, so the query tile's shared memory is free:
+      // each thread stages its head's 256 values there (rows 1040 bytes
+      // apart, conflict-free) and writes them with one bulk copy.
       tc_fence_after();
       const int64_t rh = (int64_t)r * p.H + h;
       const bool write = h < p.H;
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const bool final_out = p.n_splits == 1;
+      const bool as_bf16 = final_out && p.out_bf16;
+      const float mul = final_out ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
+      uint8_t* srow = smem + kOffQ + h * kStageRow;
 #pragma unroll 1
       for (int cb = 0; cb < 8; ++cb) {
         uint32_t ov[32];
         tmem_ld32(lane_addr + 32 * cb, ov);
         tc_wait_ld();
-        if (!write) continue;
-        if (p.n_splits == 1) {
-          if (p.out_bf16) {
-            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + rh * kDV + 256 * v + 32 * cb);
+        if (as_bf16) {
+          uint4* d = reinterpret_cast<uint4*>(srow + cb * 64);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint32_t w4[4];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w4[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
-                                                                 __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
-                w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
-              }
-              o[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q4 + 2 * e]) * mul,
+                                                               __uint_as_float(ov[8 * q4 + 2 * e + 1]) * mul);
+              w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
             }
-          } else {
-            float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + rh * kDV + 256 * v + 32 * cb);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              o[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv_l, __uint_as_float(ov[4 * q4 + 1]) * inv_l,
-                                  __uint_as_float(ov[4 * q4 + 2]) * inv_l, __uint_as_float(ov[4 * q4 + 3]) * inv_l);
+            d[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         } else {
-          const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
-          float4* o = reinterpret_cast<float4*>(p.ws_o + slot * kDV + 256 * v + 32 * cb);
+          float4* d = reinterpret_cast<float4*>(srow + cb * 128);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4)
-            o[q4] = make_float4(__uint_as_float(ov[4 * q4]), __uint_as_float(ov[4 * q4 + 1]),
-                                __uint_as_float(ov[4 * q4 + 2]), __uint_as_float(ov[4 * q4 + 3]));
+            d[q4] = make_float4(__uint_as_float(ov[4 * q4]) * mul, __uint_as_float(ov[4 * q4 + 1]) * mul,
+                                __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
         }
       }
+      if (write) {
+        fence_proxy_async_smem();
+        void* dst;
+        if (!final_out)
+          dst = p.ws_o + (((int64_t)r * p.n_splits + sp) * p.H + h) * kDV + 256 * v;
+        else if (p.out_bf16)
+          dst = reinterpret_cast<__nv_bfloat16*>(p.out) + rh * kDV + 256 * v;
+        else
+          dst = reinterpret_cast<float*>(p.out) + rh * kDV + 256 * v;
+        bulk_store_s2g(dst, smem_u32(srow), as_bf16 ? 512u : 1024u);
+        bulk_commit();
+      }
       if (write && v == 0) {
-        if (p.n_splits == 1) {
+        if (final_out) {
           if (p.lse) p.lse[rh] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
         } else {
           const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
@@ -377,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.ws_ml[2 * slot + 1] = l_run;
         }
       }
+      if (write) bulk_wait_all();  // shared memory stays valid until the copy is done
     }
   }
 
@@ -391,62 +404,72 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
-// Thread c owns columns 4c..4c+3; the split loop is unrolled so its loads are
-// in flight together.
-__global__ void __launch_bounds__(128)
+// Two CTAs of 64 threads per (row, head), one per column half; thread c owns
+// four columns and issues the loads of every split at once.
+constexpr int kMaxSplits = 32;
+__global__ void __launch_bounds__(64)
     mla_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
-  __shared__ float s_w[128];
-  __shared__ float s_red[2][4];
+  __shared__ float s_w[kMaxSplits];
+  __shared__ float s_ml[2];
   grid_dependency_wait();  // partials come from the previous kernel
   allow_dependents_launch();
-  const int64_t rh = blockIdx.x;  // row * H + head
+  const int64_t rh = blockIdx.x >> 1;  // row * H + head
+  const int half = blockIdx.x & 1;
   const int64_t r = rh / H, h = rh % H;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float m = -INFINITY, l = 0.f;
-  if ((int)threadIdx.x < n_splits) {
-    const int64_t slot = (r * n_splits + threadIdx.x) * H + h;
-    m = ws_ml[2 * slot];
-    l = ws_ml[2 * slot + 1];
+  const int c4 = half * 64 + threadIdx.x;  // float4 column of the 512
+  const float4* base = reinterpret_cast<const float4*>(ws_o + (r * n_splits * H + h) * kDV) + c4;
+  const int64_t stride4 = (int64_t)H * kDV / 4;  // between consecutive splits
+  float4 o[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s)
+    if (s < n_splits) o[s] = __ldg(base + s * stride4);
+  if (threadIdx.x < 32) {
+    const int s = threadIdx.x;
+    float m = -INFINITY, l = 0.f;
+    if (s < n_splits) {
+      const int64_t slot = (r * n_splits + s) * H + h;
+      m = ws_ml[2 * slot];
+      l = ws_ml[2 * slot + 1];
+    }
+    float M = m;
+#pragma unroll
+    for (int d = 16; d; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    float L = l * f;
+#pragma unroll
+    for (int d = 16; d; d >>= 1) L += __shfl_xor_sync(0xffffffffu, L, d);
+    s_w[s] = f;
+    if (s == 0) {
+      s_ml[0] = M;
+      s_ml[1] = L;
+    }
   }
-  float M = m;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) s_red[0][warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
-  const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
-  s_w[threadIdx.x] = f;
-  float L = l * f;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  if (lane == 0) s_red[1][warp] = L;
-  __syncthreads();
-  L = (s_red[1][0] + s_red[1][1]) + (s_red[1][2] + s_red[1][3]);
+  const float M = s_ml[0], L = s_ml[1];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-    const float4* base = reinterpret_cast<const float4*>(ws_o + (r * n_splits * H + h) * kDV) + threadIdx.x;
-    const int64_t stride4 = (int64_t)H * kDV / 4;  // between consecutive splits
-#pragma unroll 8
-    for (int s = 0; s < n_splits; ++s) {
-      const float4 o = __ldg(base + s * stride4);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < n_splits) {
       const float fs = s_w[s];
-      acc.x = fmaf(o.x, fs, acc.x);
-      acc.y = fmaf(o.y, fs, acc.y);
-      acc.z = fmaf(o.z, fs, acc.z);
-      acc.w = fmaf(o.w, fs, acc.w);
+      acc.x = fmaf(o[s].x, fs, acc.x);
+      acc.y = fmaf(o[s].y, fs, acc.y);
+      acc.z = fmaf(o[s].z, fs, acc.z);
+      acc.w = fmaf(o[s].w, fs, acc.w);
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if (out_bf16) {
-    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + rh * kDV) + 2 * threadIdx.x;
-    o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + rh * kDV)[c4] =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
   } else {
-    reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + rh * kDV)[threadIdx.x] =
+    reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + rh * kDV)[c4] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
-  if (threadIdx.x == 0 && lse) lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  if (half == 0 && threadIdx.x == 0 && lse)
+    lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace
@@ -459,6 +482,9 @@ __global__ void __launch_bounds__(128)
 // half) to cover the SMs when there are few rows, but at least
 // DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split, since every split costs one
 // query-tile load and one 128 x 512 fp32 partial.
+static_assert((DSA_MAX_TOPK + kChunk - 1) / kChunk / DSA_MLA_MIN_CHUNKS_PER_SPLIT <= kMaxSplits,
+              "the combine holds every split of a row in registers");
+
 int mla_num_splits(int n_rows, int k) {
   const int n_chunks = (k + kChunk - 1) / kChunk;
   const int sms = device_info().sm_count;
@@ -517,7 +543,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (ns > 1) {
-    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(128), 0, stream,
+    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H * 2)), dim3(64), 0, stream,
                    (const float*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
