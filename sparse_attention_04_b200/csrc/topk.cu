@@ -372,29 +372,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ============================================================================
 // Cluster variant for long rows: CS CTAs (one thread-block cluster) per row,
-// each owning a contiguous, word-aligned slice of positions.  The CTAs
-// exchange data by writing into each other's shared memory (remote stores,
-// absorbed by the next cluster barrier) in four rounds:
-//   1  every CTA sends each bin range of its 12-bit histogram to the range's
-//      owner (CTA c owns bins [c*4096/CS, (c+1)*4096/CS))
-//   2  every owner sums its range and sends it, with its total, to all CTAs;
-//      each CTA then finds bin d* (the k-th largest key's bin) locally
-//   3  every CTA marks its keys above d* in its bitmap (one warp per 32
-//      positions, via ballots) and sends its candidates (keys in bin d*) and
-//      counts to rank 0
-//   4  rank 0 fixes the exact threshold tau over all candidates and sends
-//      each CTA tau, its tie quota and its output offset
-// after which every CTA writes its kept positions independently.
+// each owning a contiguous, word-aligned slice of positions.  Two cluster
+// barriers in all:
+//   1  every CTA loads its slice (keys kept in shared memory), builds the
+//      12-bit histogram of its keys and 64 coarse sums of 64 bins each
+//   -- barrier 1 --
+//   2  every CTA reads the coarse sums of all CTAs, then the 64 fine bins of
+//      the coarse bin holding the k-th largest key (distributed shared
+//      memory), and so finds bin d* and the count of keys above it -- the
+//      same answer in every CTA
+//   3  every CTA marks its keys above bin d* in a bitmap and sends its keys
+//      in bin d* (the candidates), their count and its above-count to every
+//      CTA of the cluster
+//   -- barrier 2 --
+//   4  every CTA fixes the exact threshold tau over all candidates and its
+//      own output offset and tie quota, then writes its kept positions.
+// If any CTA has more candidates than its send buffer holds (massive ties),
+// rank 0 redoes the row with the exact digit-pass fallback.
 template <int CS>
 struct ClusterCfg {
+  static constexpr int kThreads = 512;
+  static constexpr int kWarps = kThreads / 32;
   static constexpr int kSliceMax = 131072 / CS;          // positions per CTA
   static constexpr int kSliceWords = kSliceMax / 32;
-  static constexpr int kPart = kBins12 / CS;               // bins owned per CTA
-  static constexpr int kLocalCap = 2048;                   // candidates kept per CTA
-  static constexpr int kPerSrc = 8192 / CS;                // candidates each CTA may send rank 0
-  static constexpr int kThreads = 256;
-  static constexpr int kWarps = kThreads / 32;
-  static constexpr int kWordsPerThread = kSliceWords / kThreads;
+  static constexpr int kPerSrc = 8192 / CS;                // candidates a CTA may send
+  static_assert(kSliceWords <= kThreads, "one bitmap word per thread");
+  static_assert(CS <= kWarps && CS <= 32 && 32 % CS == 0, "per-source counting and lane groups");
 };
 
 template <int CS>
@@ -402,28 +405,65 @@ struct ClusterSmem {
   using C = ClusterCfg<CS>;
   uint32_t warp_tot[32];
   uint32_t carry, sel_digit, sel_remaining, n_cand;
-  uint32_t above_count, pad0[3];
-  uint32_t tau, need_eq, eq_base, out_base, mode, pad1[3];
-  uint32_t all_tot[CS];                // every owner's bin-range total
-  uint32_t g_cnt[CS], g_above[CS];     // rank 0: candidates and above-counts per CTA
-  uint32_t cnt_gt[CS], cnt_eq[CS];     // rank 0 scratch
-  uint32_t hist[kBins12];              // local histogram, later scratch
-  uint32_t recv_hist[CS][C::kPart];    // owner: the range from every CTA
-  uint32_t all_part[kBins12];          // every CTA: the summed histogram
+  uint32_t above_local, mode, J, aboveJ;
+  uint32_t coarse[64];                 // this CTA's coarse sums (read by every CTA)
+  uint32_t tot_coarse[64];             // cluster-wide coarse sums
+  uint32_t tot_fine[64];               // cluster-wide fine bins of the chosen coarse bin
+  uint32_t g_cnt[CS], g_above[CS];     // from every CTA: candidate count, keys above d*
+  uint32_t g_off[CS + 1];              // exclusive prefix of g_cnt
+  uint32_t c_gt[CS], c_eq[CS];         // per source: candidates above / equal to tau
+  uint32_t hist[kBins12];              // 12-bit histogram of this slice, later scratch
   uint32_t bitmap[C::kSliceWords];
   uint32_t eqmap[C::kSliceWords];
-  uint32_t cand_key[C::kLocalCap];
-  uint32_t cand_pos[C::kLocalCap];
-  uint32_t keys[C::kSliceMax];
-  uint32_t g_key[CS][C::kPerSrc];      // rank 0: candidates from every CTA
+  uint32_t cand_key[C::kPerSrc];
+  uint32_t cand_pos[C::kPerSrc];
+  alignas(16) uint32_t keys[C::kSliceMax];  // written as uint4
+  uint32_t g_key[CS][C::kPerSrc];      // candidates from every CTA
 };
+
+// Over 64 bins in descending bin order (bins[63] first), finds the bin that
+// holds the `need`-th largest element.  One warp; every lane gets the answer.
+__device__ __forceinline__ void warp_select64(const uint32_t* bins, uint32_t need, int lane, int* bin,
+                                              uint32_t* above) {
+  const uint32_t c0 = bins[63 - lane], c1 = bins[31 - lane];
+  uint32_t i0 = c0, i1 = c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
+    if (lane >= o) {
+      i0 += u0;
+      i1 += u1;
+    }
+  }
+  i1 += __shfl_sync(0xffffffffu, i0, 31);
+  const unsigned b0 = __ballot_sync(0xffffffffu, i0 >= need);
+  const unsigned b1 = __ballot_sync(0xffffffffu, i1 >= need);
+  int d;
+  uint32_t ab;
+  if (b0) {
+    d = __ffs(b0) - 1;
+    ab = __shfl_sync(0xffffffffu, i0 - c0, d);
+  } else if (b1) {
+    const int l = __ffs(b1) - 1;
+    d = 32 + l;
+    ab = __shfl_sync(0xffffffffu, i1 - c1, l);
+  } else {  // fewer elements than need: cannot happen for L > k; take the lowest bin
+    d = 63;
+    ab = __shfl_sync(0xffffffffu, i1 - c1, 31);
+  }
+  *bin = 63 - d;
+  *above = ab;
+}
 
 template <int CS>
 __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
     topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B,
                         int T, int k, int32_t* __restrict__ indices, int32_t* status) {
   using Cfg = ClusterCfg<CS>;
-  constexpr int kThreads = Cfg::kThreads, kWarps = Cfg::kWarps;
+  constexpr int NT = Cfg::kThreads;
+  constexpr uint32_t kPerSrc = Cfg::kPerSrc;
+  static_assert(NT * 8 == kBins12, "coarse sums: 8 bins per thread");
+  static_assert(offsetof(ClusterSmem<CS>, keys) % 16 == 0, "16-byte key stores");
   namespace cg = cooperative_groups;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   ClusterSmem<CS>& sm = *reinterpret_cast<ClusterSmem<CS>*>(smem_raw);
@@ -439,7 +479,7 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   const int E = off[b + 1] - off[b];
   if (E < T || (int64_t)E > ld || off[b] < 0) {  // same verdict in every CTA of the cluster
     if (rank == 0) {
-      for (int j = threadIdx.x; j < k; j += kThreads) out[j] = -1;
+      for (int j = threadIdx.x; j < k; j += NT) out[j] = -1;
       if (threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
     }
     return;
@@ -448,7 +488,7 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   const float* row = scores + (int64_t)r * ld;
   if (L <= k) {
     if (rank == 0)
-      for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < L ? j : -1;
+      for (int j = threadIdx.x; j < k; j += NT) out[j] = j < L ? j : -1;
     return;
   }
   // slice of this CTA, word aligned (the host sends only rows of <= 131072 positions here)
@@ -457,18 +497,18 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   const int n = s_hi - s_lo;
   const int n_words = (n + 31) >> 5;
 
-  // ---- round 1: keys of the slice, local histogram, ranges to their owners
-  for (int i = threadIdx.x; i < kBins12; i += kThreads) sm.hist[i] = 0;
+  // ---- 1: keys and 12-bit histogram of the slice, coarse sums
+  for (int i = threadIdx.x; i < kBins12; i += NT) sm.hist[i] = 0;
   if (threadIdx.x == 0) {
     sm.n_cand = 0;
-    sm.above_count = 0;
+    sm.above_local = 0;
   }
   __syncthreads();
   {
     const float4* r4 = reinterpret_cast<const float4*>(row + s_lo);  // s_lo is a multiple of 32
     uint4* k4 = reinterpret_cast<uint4*>(sm.keys);
     const int n4 = n >> 2;
-    for (int i4 = threadIdx.x; i4 < n4; i4 += kThreads) {
+    for (int i4 = threadIdx.x; i4 < n4; i4 += NT) {
       const float4 v = __ldg(r4 + i4);
       const uint4 kk = make_uint4(float_order_key(v.x), float_order_key(v.y), float_order_key(v.z),
                                   float_order_key(v.w));
@@ -478,69 +518,72 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
       atomicAdd(&sm.hist[kk.z >> 20], 1u);
       atomicAdd(&sm.hist[kk.w >> 20], 1u);
     }
-    for (int s = 4 * n4 + threadIdx.x; s < n; s += kThreads) {
+    for (int s = 4 * n4 + threadIdx.x; s < n; s += NT) {
       const uint32_t key = float_order_key(__ldg(row + s_lo + s));
       sm.keys[s] = key;
       atomicAdd(&sm.hist[key >> 20], 1u);
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kBins12; i += kThreads) {
-    const int q = i / Cfg::kPart;
-    cluster.map_shared_rank(&sm.recv_hist[0][0], q)[rank * Cfg::kPart + (i - q * Cfg::kPart)] = sm.hist[i];
-  }
-  cluster.sync();  // 1
-
-  // ---- round 2: owners sum their range and send it to everyone
   {
-    uint32_t mine = 0;
-    for (int i = threadIdx.x; i < Cfg::kPart; i += kThreads) {
-      uint32_t sum = 0;
+    uint32_t v = 0;
 #pragma unroll
-      for (int q = 0; q < CS; ++q) sum += sm.recv_hist[q][i];
-      mine += sum;
+    for (int j = 0; j < 8; ++j) v += sm.hist[8 * threadIdx.x + j];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    if ((threadIdx.x & 7) == 0) sm.coarse[threadIdx.x >> 3] = v;
+  }
+  cluster.sync();  // 1: every histogram and coarse sum is complete
+
+  // ---- 2: bin d* from the cluster-wide histogram (the same in every CTA).
+  // Entry e = j * CS + q: bin j of CTA q; the CS lanes of a group sum over q.
+  for (int e = threadIdx.x; e < 64 * CS; e += NT) {
+    const int j = e / CS, q = e % CS;
+    uint32_t v = cluster.map_shared_rank(sm.coarse, q)[j];
 #pragma unroll
-      for (int q = 0; q < CS; ++q) cluster.map_shared_rank(sm.all_part, q)[rank * Cfg::kPart + i] = sum;
-    }
-    uint32_t tot;
-    block_excl_scan<kThreads>(mine, sm, &tot);
-    if (threadIdx.x < CS) cluster.map_shared_rank(sm.all_tot, (int)threadIdx.x)[rank] = tot;
+    for (int o = CS / 2; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (q == 0) sm.tot_coarse[j] = v;
   }
-  cluster.sync();  // 2
-
-  // bin d* holding the k-th largest key: all data is local now
-  uint32_t dstar, need_in_bin;
-  {
-    __shared__ uint32_t s_owner, s_above;
-    if (threadIdx.x == 0) {  // owners in descending bin order: rank CS-1 holds the highest bins
-      uint32_t above = 0;
-      int owner = 0;
-      for (int q = CS - 1; q >= 0; --q) {
-        if (above + sm.all_tot[q] >= (uint32_t)k) {
-          owner = q;
-          break;
-        }
-        above += sm.all_tot[q];
-      }
-      s_owner = (uint32_t)owner;
-      s_above = above;
+  __syncthreads();
+  if (warp == 0) {
+    int J;
+    uint32_t ab;
+    warp_select64(sm.tot_coarse, (uint32_t)k, lane, &J, &ab);
+    if (lane == 0) {
+      sm.J = (uint32_t)J;
+      sm.aboveJ = ab;
     }
-    __syncthreads();
-    const int owner = (int)s_owner;
-    for (int i = threadIdx.x; i < 1024; i += kThreads)
-      sm.hist[i] = i < Cfg::kPart ? sm.all_part[owner * Cfg::kPart + i] : 0u;
-    __syncthreads();
-    select_bin<kThreads>(sm, sm.hist, 1024, (uint32_t)k - s_above);
-    dstar = (uint32_t)(owner * Cfg::kPart) + sm.sel_digit;
-    need_in_bin = sm.sel_remaining;
   }
+  __syncthreads();
+  const uint32_t J = sm.J, aboveJ = sm.aboveJ;
+  for (int e = threadIdx.x; e < 64 * CS; e += NT) {
+    const int j = e / CS, q = e % CS;
+    uint32_t v = cluster.map_shared_rank(sm.hist, q)[64 * J + j];
+#pragma unroll
+    for (int o = CS / 2; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (q == 0) sm.tot_fine[j] = v;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int jf;
+    uint32_t ab;
+    warp_select64(sm.tot_fine, (uint32_t)k - aboveJ, lane, &jf, &ab);
+    if (lane == 0) {
+      sm.sel_digit = 64 * J + (uint32_t)jf;
+      sm.sel_remaining = (uint32_t)k - aboveJ - ab;
+    }
+  }
+  __syncthreads();
+  const uint32_t dstar = sm.sel_digit;
+  const uint32_t need_in_bin = sm.sel_remaining;  // keys of bin d* that are kept (>= 1)
 
-  // ---- round 3: bitmap of keys above d*, candidates in d*, counts to rank 0
+  // ---- 3: bitmap of keys above d*, candidates in d*, sent to every CTA
   {
-    uint32_t above_local = 0;
-    for (int w = warp; w < Cfg::kSliceWords; w += kWarps) {
+    uint32_t above = 0;
+    for (int w = warp; w < n_words; w += Cfg::kWarps) {
       const int s = 32 * w + lane;
-      const bool valid = w < n_words && s < n;
+      const bool valid = s < n;
       const uint32_t key = valid ? sm.keys[s] : 0u;
       const uint32_t bin = key >> 20;
       const uint32_t up = __ballot_sync(0xffffffffu, valid && bin > dstar);
@@ -551,7 +594,7 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
         base = __shfl_sync(0xffffffffu, base, 0);
         if (valid && bin == dstar) {
           const uint32_t slot = base + __popc(cand & ((1u << lane) - 1u));
-          if (slot < (uint32_t)Cfg::kLocalCap) {
+          if (slot < kPerSrc) {
             sm.cand_key[slot] = key;
             sm.cand_pos[slot] = (uint32_t)s;
           }
@@ -561,132 +604,124 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
         sm.bitmap[w] = up;
         sm.eqmap[w] = 0;
       }
-      above_local += __popc(up);
+      above += __popc(up);
     }
-    if (lane == 0 && above_local) atomicAdd(&sm.above_count, above_local);
+    for (int w = n_words + threadIdx.x; w < Cfg::kSliceWords; w += NT) {
+      sm.bitmap[w] = 0;
+      sm.eqmap[w] = 0;
+    }
+    if (lane == 0 && above) atomicAdd(&sm.above_local, above);
     __syncthreads();
     const uint32_t nc = sm.n_cand;
-    ClusterSmem<CS>* r0 = cluster.map_shared_rank(&sm, 0);
-    const bool fits = nc <= (uint32_t)Cfg::kPerSrc;
-    if (fits)
-      for (uint32_t c = threadIdx.x; c < nc; c += kThreads) r0->g_key[rank][c] = sm.cand_key[c];
-    if (threadIdx.x == 0) {
-      r0->g_cnt[rank] = fits ? nc : 0xFFFFFFFFu;  // overflow marker
-      r0->g_above[rank] = sm.above_count;
+    const bool fits = nc <= kPerSrc;
+    if (fits && nc > 0) {
+      for (uint32_t e = threadIdx.x; e < nc * CS; e += NT) {
+        const uint32_t q = e / nc, c = e - q * nc;
+        cluster.map_shared_rank(&sm, (int)q)->g_key[rank][c] = sm.cand_key[c];
+      }
+    }
+    if (threadIdx.x < CS) {
+      ClusterSmem<CS>* dst = cluster.map_shared_rank(&sm, (int)threadIdx.x);
+      dst->g_cnt[rank] = fits ? nc : 0xFFFFFFFFu;  // overflow marker
+      dst->g_above[rank] = sm.above_local;
     }
   }
-  cluster.sync();  // 3
+  cluster.sync();  // 2: no remote shared-memory access after this point
 
-  // ---- round 4: rank 0 fixes the exact threshold and every CTA's offsets
-  if (rank == 0) {
-    __shared__ uint32_t s_goff[CS + 1], s_mode;
-    if (threadIdx.x == 0) {
-      uint32_t total = 0, bad = 0;
-      for (int q = 0; q < CS; ++q) {
-        bad |= sm.g_cnt[q] == 0xFFFFFFFFu;
-        s_goff[q] = total;
-        total += bad ? 0u : sm.g_cnt[q];
-      }
-      s_goff[CS] = total;
-      s_mode = bad ? 1u : 0u;
+  // ---- 4: exact threshold tau over every candidate, this CTA's offsets, output
+  if (threadIdx.x == 0) {
+    uint32_t tot = 0, bad = 0;
+    for (int q = 0; q < CS; ++q) {
+      sm.g_off[q] = tot;
+      if (sm.g_cnt[q] == 0xFFFFFFFFu) bad = 1;
+      else tot += sm.g_cnt[q];
     }
-    if (threadIdx.x < CS) sm.cnt_gt[threadIdx.x] = sm.cnt_eq[threadIdx.x] = 0;
-    __syncthreads();
-    if (s_mode == 0) {
-      uint32_t prefix = dstar << 20, pmask = 0xFFF00000u, remaining = need_in_bin;
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        const int shift = pass == 0 ? 10 : 0;
-        for (int i = threadIdx.x; i < 1024; i += kThreads) sm.hist[i] = 0;
-        __syncthreads();
-        for (int q = 0; q < CS; ++q)
-          for (uint32_t c = threadIdx.x; c < sm.g_cnt[q]; c += kThreads) {
-            const uint32_t key = sm.g_key[q][c];
-            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
-          }
-        __syncthreads();
-        select_bin<kThreads>(sm, sm.hist, 1024, remaining);
-        prefix |= sm.sel_digit << shift;
-        pmask |= 1023u << shift;
-        remaining = sm.sel_remaining;
-        __syncthreads();
-      }
-      const uint32_t tau = prefix, need_eq = remaining;
-      for (int q = 0; q < CS; ++q)
-        for (uint32_t c = threadIdx.x; c < sm.g_cnt[q]; c += kThreads) {
-          const uint32_t key = sm.g_key[q][c];
-          if (key > tau) atomicAdd(&sm.cnt_gt[q], 1u);
-          else if (key == tau) atomicAdd(&sm.cnt_eq[q], 1u);
-        }
-      __syncthreads();
-      if (threadIdx.x < CS) {
-        const int q = (int)threadIdx.x;
-        uint32_t eq_base = 0, out_base = 0;
-        for (int p = 0; p < q; ++p) {
-          const uint32_t taken = eq_base >= need_eq ? 0u : min(sm.cnt_eq[p], need_eq - eq_base);
-          eq_base += sm.cnt_eq[p];
-          out_base += sm.g_above[p] + sm.cnt_gt[p] + taken;
-        }
-        ClusterSmem<CS>* dst = cluster.map_shared_rank(&sm, q);
-        dst->tau = tau;
-        dst->need_eq = need_eq;
-        dst->eq_base = eq_base;
-        dst->out_base = out_base;
-        dst->mode = 0;
-      }
-    } else if (threadIdx.x < CS) {
-      cluster.map_shared_rank(&sm, (int)threadIdx.x)->mode = 1;
-    }
+    sm.g_off[CS] = tot;
+    sm.mode = bad;
   }
-  cluster.sync();  // 4: no remote shared-memory access after this point
-
-  if (sm.mode == 1) {  // a CTA had too many keys in bin d*: rank 0 redoes the row alone
-    if (rank == 0) radix_select_fallback<kThreads>(sm, sm.keys, Cfg::kSliceMax, row, L, k, out);
+  __syncthreads();
+  if (sm.mode) {  // a CTA had too many keys in bin d*: rank 0 redoes the row alone
+    if (rank == 0) radix_select_fallback<NT>(sm, sm.keys, Cfg::kSliceMax, row, L, k, out);
     return;
   }
-  const uint32_t tau = sm.tau, need_eq = sm.need_eq;
-  const uint32_t n_cand = min(sm.n_cand, (uint32_t)Cfg::kLocalCap);
-  for (uint32_t c = threadIdx.x; c < n_cand; c += kThreads) {
+  const uint32_t n_all = sm.g_off[CS];
+  uint32_t prefix = dstar << 20, pmask = 0xFFF00000u, remaining = need_in_bin;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    for (int i = threadIdx.x; i < 1024; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+    for (uint32_t c = threadIdx.x; c < n_all; c += NT) {
+      int q = 0;  // source of dense index c: the last q with g_off[q] <= c
+#pragma unroll
+      for (int step = CS / 2; step; step >>= 1)
+        if (q + step < CS && sm.g_off[q + step] <= c) q += step;
+      const uint32_t key = sm.g_key[q][c - sm.g_off[q]];
+      if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
+    }
+    __syncthreads();
+    select_bin<NT>(sm, sm.hist, 1024, remaining);
+    prefix |= sm.sel_digit << shift;
+    pmask |= 1023u << shift;
+    remaining = sm.sel_remaining;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix, need_eq = remaining;
+  if (warp < CS) {  // per source: candidates above and equal to tau
+    const uint32_t cnt = sm.g_cnt[warp];
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t i = lane; i < cnt; i += 32) {
+      const uint32_t key = sm.g_key[warp][i];
+      gt += key > tau;
+      eq += key == tau;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+      sm.c_gt[warp] = gt;
+      sm.c_eq[warp] = eq;
+    }
+  }
+  __syncthreads();
+  uint32_t out_base = 0, eq_base = 0;  // what the lower slices keep
+  for (int q = 0; q < rank; ++q) {
+    const uint32_t taken = eq_base >= need_eq ? 0u : min(sm.c_eq[q], need_eq - eq_base);
+    eq_base += sm.c_eq[q];
+    out_base += sm.g_above[q] + sm.c_gt[q] + taken;
+  }
+  for (uint32_t c = threadIdx.x; c < sm.n_cand; c += NT) {
     const uint32_t key = sm.cand_key[c], s = sm.cand_pos[c];
     if (key > tau) atomicOr(&sm.bitmap[s >> 5], 1u << (s & 31));
     else if (key == tau) atomicOr(&sm.eqmap[s >> 5], 1u << (s & 31));
   }
   __syncthreads();
   {  // keys equal to tau: keep those whose rank over the whole row is below need_eq
-    const int w0 = threadIdx.x * Cfg::kWordsPerThread;
-    uint32_t cnt = 0;
-#pragma unroll
-    for (int j = 0; j < Cfg::kWordsPerThread; ++j) cnt += __popc(sm.eqmap[w0 + j]);
+    const int w = threadIdx.x;
+    uint32_t bits = w < Cfg::kSliceWords ? sm.eqmap[w] : 0u;
     uint32_t tot;
-    uint32_t rk = sm.eq_base + block_excl_scan<kThreads>(cnt, sm, &tot);
-#pragma unroll
-    for (int j = 0; j < Cfg::kWordsPerThread; ++j) {
-      uint32_t bits = sm.eqmap[w0 + j], keep = 0;
-      while (bits && rk < need_eq) {
-        const uint32_t low = bits & (0u - bits);
-        keep |= low;
-        bits ^= low;
-        ++rk;
-      }
-      if (keep) sm.bitmap[w0 + j] |= keep;
+    uint32_t rk = eq_base + block_excl_scan<NT>((uint32_t)__popc(bits), sm, &tot);
+    uint32_t keep = 0;
+    while (bits && rk < need_eq) {
+      const uint32_t low = bits & (0u - bits);
+      keep |= low;
+      bits ^= low;
+      ++rk;
     }
+    if (keep) sm.bitmap[w] |= keep;
   }
   __syncthreads();
-  {  // ascending output of this slice at its offset
-    const int w0 = threadIdx.x * Cfg::kWordsPerThread;
-    uint32_t cnt = 0;
-#pragma unroll
-    for (int j = 0; j < Cfg::kWordsPerThread; ++j) cnt += __popc(sm.bitmap[w0 + j]);
+  {  // ascending output of this slice at its offset: one bitmap word per thread
+    const int w = threadIdx.x;
+    uint32_t bits = w < Cfg::kSliceWords ? sm.bitmap[w] : 0u;
     uint32_t tot;
-    uint32_t pos = sm.out_base + block_excl_scan<kThreads>(cnt, sm, &tot);
-#pragma unroll
-    for (int j = 0; j < Cfg::kWordsPerThread; ++j) {
-      uint32_t bits = sm.bitmap[w0 + j];
-      while (bits) {
-        const int bb = __ffs(bits) - 1;
-        bits &= bits - 1;
-        out[pos++] = s_lo + 32 * (w0 + j) + bb;
-      }
+    uint32_t pos = out_base + block_excl_scan<NT>((uint32_t)__popc(bits), sm, &tot);
+    while (bits) {
+      const int bb = __ffs(bits) - 1;
+      bits &= bits - 1;
+      out[pos++] = s_lo + 32 * w + bb;
     }
   }
 }
