@@ -95,10 +95,10 @@ size_t dsa_sparse_mla_workspace_size(int B, int T, int H, int k) {
   return mla_workspace_bytes(B * T, H, k);
 }
 
-int dsa_sparse_mla(const void* q, const void* kv, const int32_t* offsets, const int32_t* indices,
-                   int B, int T, int H, int k, float scale, int64_t kv_rows, void* out,
-                   int out_dtype, float* lse, void* workspace, size_t ws_bytes,
-                   int32_t* dev_status, void* stream) {
+namespace {
+int sparse_mla_call(const void* q, const void* kv, const int32_t* offsets, const int32_t* indices, int B, int T,
+                    int H, int k, float scale, int64_t kv_rows, void* out, int out_dtype, float* lse,
+                    void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool early_inputs) {
   if (int rc = check_rows(B, T)) return rc;
   if (!q || !kv || !offsets || !indices || !out) return DSA_ERR_INVALID_ARG;
   if (H < 1 || k < 1 || k > DSA_MAX_TOPK) return DSA_ERR_INVALID_ARG;
@@ -109,8 +109,18 @@ int dsa_sparse_mla(const void* q, const void* kv, const int32_t* offsets, const 
     return DSA_ERR_INVALID_ARG;
   const size_t need = mla_workspace_bytes(B * T, H, k);
   if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return DSA_ERR_WORKSPACE;
-  MlaArgs a{q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out, out_dtype, lse, workspace, ws_bytes, dev_status};
+  MlaArgs a{q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out, out_dtype, lse, workspace, ws_bytes, dev_status,
+            early_inputs};
   return launch_sparse_mla(a, reinterpret_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int dsa_sparse_mla(const void* q, const void* kv, const int32_t* offsets, const int32_t* indices,
+                   int B, int T, int H, int k, float scale, int64_t kv_rows, void* out,
+                   int out_dtype, float* lse, void* workspace, size_t ws_bytes,
+                   int32_t* dev_status, void* stream) {
+  return sparse_mla_call(q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out, out_dtype, lse, workspace,
+                         ws_bytes, dev_status, stream, false);
 }
 
 int dsa_decode_step_workspace_layout(int B, int max_end_pos, int k, int H, size_t* scores_off,
@@ -157,8 +167,8 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
   if (rc) return rc;
   rc = dsa_topk(scores, ld, offsets, B, 1, k, indices, dev_status, stream);
   if (rc) return rc;
-  return dsa_sparse_mla(q, kv, offsets, indices, B, 1, H, k, scale, kv_rows, out, out_dtype, lse,
-                        ws + m_off, ws_bytes - m_off, dev_status, stream);
+  return sparse_mla_call(q, kv, offsets, indices, B, 1, H, k, scale, kv_rows, out, out_dtype, lse, ws + m_off,
+                         ws_bytes - m_off, dev_status, stream, true);
 }
 
 }  // extern "C"

@@ -70,6 +70,11 @@ struct MlaArgs {
   void* workspace;
   size_t ws_bytes;
   int32_t* status;
+  // The step's inputs (q, offsets) were complete before the preceding kernel
+  // in the stream started (true inside dsa_decode_step, whose first kernel
+  // waited for them): the kernel may then read them before its dependency
+  // wait.  Standalone calls wait first.
+  bool early_inputs;
 };
 int mla_num_splits(int n_rows, int k);
 size_t mla_workspace_bytes(int n_rows, int H, int k);

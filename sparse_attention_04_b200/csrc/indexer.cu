@@ -82,7 +82,7 @@ __device__ __forceinline__ int seg_len(const int32_t* __restrict__ off, int T, i
 }
 
 struct SmemMisc {
-  int seg0, kt0, count, abort, tmem_base, bad, pad[10];
+  int abort, tmem_base, pad[14];
 };
 
 // 64-head weighted ReLU sum of one key for one query: sum_h w[h]*max(0, d[h]),
@@ -103,6 +103,66 @@ __device__ __forceinline__ float head_sum64(const uint32_t (&v0)[32], const uint
     a[2 * j + 1] = __ffma2_rn(x23, make_float2(w4.z, w4.w), a[2 * j + 1]);
   }
   return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+}
+
+// This CTA's range of work (warp-collective; every lane gets the result).
+// The offsets are validated first.  Segment (query block) s costs
+// SEG_COST + len_s units, its tiles being the last len_s of them; the CTA
+// takes units [lo, hi) of the total and scores the tiles among them, which
+// are contiguous in the flat tile list.
+struct Split {
+  int seg0, kt0, count;
+  bool bad;
+};
+
+template <int NQ, int SEG_COST>
+__device__ Split find_split(const int32_t* __restrict__ off, int B, int T, int64_t kv_rows, int64_t ld, int QB,
+                            int nseg, int lane) {
+  bool bad = false;
+  for (int b = lane; b < B; b += 32) {
+    const int E = off[b + 1] - off[b];
+    bad |= (off[b] < 0) || (E < T) || ((int64_t)E > ld);
+  }
+  if (lane == 0) bad |= ((int64_t)off[B] > kv_rows);
+  bad = __any_sync(0xffffffffu, bad);
+  Split r{0, 0, 0, bad};
+  if (bad) return r;
+  int64_t total = 0;
+  for (int base = 0; base < nseg; base += 32) {
+    const int seg = base + lane;
+    int64_t u = seg < nseg ? seg_len<NQ>(off, T, QB, seg) + SEG_COST : 0;
+    for (int o = 16; o; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+    total += u;
+  }
+  const int64_t lo = total * blockIdx.x / gridDim.x;
+  const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+  int64_t count = 0, acc = 0;
+  bool found = false;
+  for (int base = 0; base < nseg && acc < hi; base += 32) {
+    const int seg = base + lane;
+    const int len = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
+    const int64_t u = seg < nseg ? len + SEG_COST : 0;
+    int64_t incl = u;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int64_t tile_lo = acc + incl - len, tile_hi = acc + incl;  // this segment's tile units
+    const int64_t ov_lo = max(tile_lo, lo), ov_hi = min(tile_hi, hi);
+    int64_t ov = ov_hi > ov_lo ? ov_hi - ov_lo : 0;
+    const unsigned m = __ballot_sync(0xffffffffu, ov > 0);
+    if (!found && m) {
+      const int src = __ffs(m) - 1;
+      r.seg0 = __shfl_sync(0xffffffffu, seg, src);
+      r.kt0 = (int)__shfl_sync(0xffffffffu, ov_lo - tile_lo, src);
+      found = true;
+    }
+    for (int o = 16; o; o >>= 1) ov += __shfl_xor_sync(0xffffffffu, ov, o);
+    count += ov;
+    acc += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  r.count = found ? (int)count : 0;
+  return r;
 }
 
 template <int NQ, bool FP8>
@@ -151,75 +211,21 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
     tmem_alloc(sbase + C::OFF_MISC + offsetof(SmemMisc, tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
-  grid_dependency_wait();
-  allow_dependents_launch();
-
-  // ---- validate offsets and find this CTA's balanced range of work units.
-  // Segment (query block) s costs SEG_COST + len_s units; its tiles are the
-  // last len_s of them.  The CTA takes units [lo, hi) and scores the tiles
-  // among them, which are contiguous in the flat tile list.
-  if (warp == 0) {
-    bool bad = false;
-    for (int b = lane; b < B; b += 32) {
-      const int E = off[b + 1] - off[b];
-      bad |= (off[b] < 0) || (E < T) || ((int64_t)E > ld);
-    }
-    if (lane == 0) bad |= ((int64_t)off[B] > kv_rows);
-    bad = __any_sync(0xffffffffu, bad);
-    int64_t total = 0;
-    if (!bad)
-      for (int base = 0; base < nseg; base += 32) {
-        const int seg = base + lane;
-        int64_t u = seg < nseg ? seg_len<NQ>(off, T, QB, seg) + C::SEG_COST : 0;
-        for (int o = 16; o; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-        total += u;
-      }
-    const int64_t lo = total * blockIdx.x / gridDim.x;
-    const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
-    int seg0 = 0, kt0 = 0;
-    int64_t count = 0;
-    bool found = false;
-    int64_t acc = 0;
-    for (int base = 0; base < nseg && acc < hi && !bad; base += 32) {
-      const int seg = base + lane;
-      const int len = seg < nseg ? seg_len<NQ>(off, T, QB, seg) : 0;
-      const int64_t u = seg < nseg ? len + C::SEG_COST : 0;
-      int64_t incl = u;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int64_t tile_lo = acc + incl - len, tile_hi = acc + incl;  // this segment's tile units
-      const int64_t ov_lo = max(tile_lo, lo), ov_hi = min(tile_hi, hi);
-      int64_t ov = ov_hi > ov_lo ? ov_hi - ov_lo : 0;
-      const unsigned m = __ballot_sync(0xffffffffu, ov > 0);
-      if (!found && m) {
-        const int src = __ffs(m) - 1;
-        seg0 = __shfl_sync(0xffffffffu, seg, src);
-        kt0 = (int)__shfl_sync(0xffffffffu, ov_lo - tile_lo, src);
-        found = true;
-      }
-      for (int o = 16; o; o >>= 1) ov += __shfl_xor_sync(0xffffffffu, ov, o);
-      count += ov;
-      acc += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) {
-      misc->seg0 = seg0;
-      misc->kt0 = kt0;
-      misc->count = (bad || !found) ? 0 : (int)count;
-      misc->abort = 0;
-      misc->bad = bad ? 1 : 0;
-      if (bad && blockIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
-    }
-  }
+  if (threadIdx.x == 0) misc->abort = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(misc->tmem_base);
-  const int count = misc->count;
+  grid_dependency_wait();
+  allow_dependents_launch();
+
+  // Every role warp finds the CTA's work range itself (no block-wide sync).
+  const Split sp = find_split<NQ, C::SEG_COST>(off, B, T, kv_rows, ld, QB, nseg, lane);
+  if (sp.bad && blockIdx.x == 0 && threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
+  const int count = sp.count;
 
   // Walk of the CTA's items, identical in every role.
-  int seg = misc->seg0, kt = misc->kt0;
+  int seg = sp.seg0, kt = sp.kt0;
   int len = count > 0 ? seg_len<NQ>(off, T, QB, seg) : 0;
 
   if (warp == C::PRODUCER) {
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
     // Written 512 bytes per step, a few steps after each load (decode rows
     // have nothing to fill).
     const int64_t n_rows = (int64_t)B * T;
-    int64_t f_r = (T > 1 && !misc->bad) ? (int64_t)blockIdx.x : n_rows;
+    int64_t f_r = (T > 1 && !sp.bad) ? (int64_t)blockIdx.x : n_rows;
     int64_t f_pos = 0, f_end = 0;
     float* f_row = scores;
     auto fill = [&](int steps) {
@@ -270,15 +276,6 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
             tma_load_2d(sbase + C::OFF_Q + qs * C::Q_BYTES + bx * (C::N * 128), &tm_q,
                         bx * (FP8 ? 128 : 64), y, q_full(qs));
         }
-        // per-head weights of this query block, for the epilogue (staged while
-        // the copies fly; the second arrival on q_full publishes them)
-        float* wd = w_s + qs * C::N;
-        for (int i = lane; i < C::N; i += 32) {
-          const int t = qb * NQ + i / kHI;
-          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full(qs));
       }
       const int st = item % C::KSTAGES;
       bool ok = mbar_wait(k_empty(st), ((item / C::KSTAGES) & 1) ^ 1, abort, kWaitLimitNs);
@@ -289,6 +286,18 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
         for (int bx = 0; bx < C::BOXES; ++bx)
           tma_load_2d(sbase + C::OFF_K + st * C::KT_BYTES + bx * 16384, &tm_k,
                       bx * (FP8 ? 128 : 64), y, k_full(st));
+      }
+      if (item == 0 || kt == 0) {
+        // per-head weights of this query block, for the epilogue, staged while
+        // both copies fly; the second arrival on q_full publishes them
+        const int qs = qord & 1;
+        float* wd = w_s + qs * C::N;
+        for (int i = lane; i < C::N; i += 32) {
+          const int t = qb * NQ + i / kHI;
+          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full(qs));
       }
       issued = item + 1;
       fill(4);

@@ -117,6 +117,9 @@ __device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until every committed bulk group of this thread has finished reading
+// its shared-memory source (the global writes complete by kernel end).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- cp.async
 
@@ -271,6 +274,16 @@ __device__ __forceinline__ void grid_dependency_wait() {
 __device__ __forceinline__ void allow_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// ---------------------------------------------------------------- clusters
+
+// Split cluster barrier: arrive (no memory ordering) ... wait.  Used once at
+// kernel start so that no CTA touches another's shared memory before every
+// CTA of the cluster has started.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- misc
 

@@ -76,6 +76,7 @@ struct MlaParams {
   float* ws_o;   // [rows][splits][H][512]   (n_splits > 1)
   float* ws_ml;  // [rows][splits][H][2]
   int32_t* status;
+  int early_inputs;  // q and offsets may be read before the dependency wait
 };
 
 __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 && idx < E; }
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &misc->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!p.early_inputs) grid_dependency_wait();  // q and the offsets may come from the previous kernel
   const int v = blockIdx.x & 1;
   const int sp = (blockIdx.x >> 1) % p.n_splits;
   const int r = (blockIdx.x >> 1) / p.n_splits;
@@ -108,9 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks_total = (p.k + kChunk - 1) / kChunk;
   const int c_end = min(c_begin + p.cps, n_chunks_total);
 
-  // ---- prologue: barriers, TMEM, and the query tile (q is an input of the
-  // whole step, written before the indexer ran), overlapping the previous
-  // kernel's tail.
+  // ---- prologue: barriers, TMEM, and the query tile, overlapping the
+  // previous kernel's tail when the inputs are known to be complete.
   if (threadIdx.x == 0) {
     misc->last_valid = -1;
     misc->abort = 0;
@@ -238,22 +239,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
     // the two groups run independently, so both stages are in flight from
     // the start and a group waits only for its own copies before it signals.
+    // Each warp copies 16 whole rows, one row at a time, so every copy
+    // instruction reads 512 contiguous bytes of a row.
     const int pt = threadIdx.x - 128;
-    const int grp = pt >> 6, gt = pt & 63;
-    const int jr = gt >> 1, part = gt & 1;
+    const int grp = pt >> 6, gw = (pt >> 5) & 1;
     const __nv_bfloat16* kv = p.kv;
     for (int i = grp; i < n_my; i += 2) {
       const int st = i & 1;
       if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
-      const int pos = (c_begin + i) * kChunk + jr;
-      const int32_t id = pos < p.k ? idx_row[pos] : -1;
-      const bool valid = index_ok(id, E);
-      const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
-      const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
-#pragma unroll 4
-      for (int c = part; c < kDQK / 8; c += 2) {
-        const int kb = c >> 3, cc = c & 7;
-        cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+      int32_t my_id = -1;
+      if (lane < 16) {
+        const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
+        my_id = pos < p.k ? idx_row[pos] : -1;
+      }
+#pragma unroll 2
+      for (int rr = 0; rr < 16; ++rr) {
+        const int jr = gw * 16 + rr;
+        const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
+        const bool valid = index_ok(id, E);
+        const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
+        const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
+          if (c < kDQK / 8) {
+            const int kb = c >> 3, cc = c & 7;
+            cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+          }
+        }
       }
       cp_async_commit();
       cp_async_wait<0>();
@@ -343,10 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mul = final_out ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
       uint8_t* srow = smem + kOffQ + h * kStageRow;
 #pragma unroll 1
-      for (int cb = 0; cb < 8; ++cb) {
-        uint32_t ov[32];
-        tmem_ld32(lane_addr + 32 * cb, ov);
+      for (int cb2 = 0; cb2 < 8; cb2 += 2) {
+        uint32_t ovp[2][32];
+        tmem_ld32(lane_addr + 32 * cb2, ovp[0]);
+        tmem_ld32(lane_addr + 32 * cb2 + 32, ovp[1]);
         tc_wait_ld();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+        const int cb = cb2 + half;
+        const uint32_t (&ov)[32] = ovp[half];
         if (as_bf16) {
           uint4* d = reinterpret_cast<uint4*>(srow + cb * 64);
 #pragma unroll
@@ -366,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q4 = 0; q4 < 8; ++q4)
             d[q4] = make_float4(__uint_as_float(ov[4 * q4]) * mul, __uint_as_float(ov[4 * q4 + 1]) * mul,
                                 __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
+        }
         }
       }
       if (write) {
@@ -389,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.ws_ml[2 * slot + 1] = l_run;
         }
       }
-      if (write) bulk_wait_all();  // shared memory stays valid until the copy is done
+      if (write) bulk_wait_read();  // shared memory stays valid until the copy has read it
     }
   }
 
@@ -406,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
 // Two CTAs of 64 threads per (row, head), one per column half; thread c owns
 // four columns and issues the loads of every split at once.
-constexpr int kMaxSplits = 32;
+constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(64)
     mla_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
@@ -420,27 +439,35 @@ __global__ void __launch_bounds__(64)
   const int c4 = half * 64 + threadIdx.x;  // float4 column of the 512
   const float4* base = reinterpret_cast<const float4*>(ws_o + (r * n_splits * H + h) * kDV) + c4;
   const int64_t stride4 = (int64_t)H * kDV / 4;  // between consecutive splits
-  float4 o[kMaxSplits];
+  // the first 32 splits' loads are issued before the weights are known
+  float4 o[32];
 #pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s)
+  for (int s = 0; s < 32; ++s)
     if (s < n_splits) o[s] = __ldg(base + s * stride4);
   if (threadIdx.x < 32) {
-    const int s = threadIdx.x;
-    float m = -INFINITY, l = 0.f;
-    if (s < n_splits) {
-      const int64_t slot = (r * n_splits + s) * H + h;
-      m = ws_ml[2 * slot];
-      l = ws_ml[2 * slot + 1];
+    const int s0 = threadIdx.x, s1 = threadIdx.x + 32;
+    float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
+    if (s0 < n_splits) {
+      const int64_t slot = (r * n_splits + s0) * H + h;
+      m0 = ws_ml[2 * slot];
+      l0 = ws_ml[2 * slot + 1];
     }
-    float M = m;
+    if (s1 < n_splits) {
+      const int64_t slot = (r * n_splits + s1) * H + h;
+      m1 = ws_ml[2 * slot];
+      l1 = ws_ml[2 * slot + 1];
+    }
+    float M = fmaxf(m0, m1);
 #pragma unroll
     for (int d = 16; d; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
-    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    float L = l * f;
+    const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
+    const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
+    float L = l0 * f0 + l1 * f1;
 #pragma unroll
     for (int d = 16; d; d >>= 1) L += __shfl_xor_sync(0xffffffffu, L, d);
-    s_w[s] = f;
-    if (s == 0) {
+    s_w[s0] = f0;
+    s_w[s1] = f1;
+    if (s0 == 0) {
       s_ml[0] = M;
       s_ml[1] = L;
     }
@@ -449,13 +476,28 @@ __global__ void __launch_bounds__(64)
   const float M = s_ml[0], L = s_ml[1];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s) {
+  for (int s = 0; s < 32; ++s) {
     if (s < n_splits) {
       const float fs = s_w[s];
       acc.x = fmaf(o[s].x, fs, acc.x);
       acc.y = fmaf(o[s].y, fs, acc.y);
       acc.z = fmaf(o[s].z, fs, acc.z);
       acc.w = fmaf(o[s].w, fs, acc.w);
+    }
+  }
+  if (n_splits > 32) {  // the second group of splits
+#pragma unroll
+    for (int s = 0; s < 32; ++s)
+      if (32 + s < n_splits) o[s] = __ldg(base + (32 + s) * stride4);
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+      if (32 + s < n_splits) {
+        const float fs = s_w[32 + s];
+        acc.x = fmaf(o[s].x, fs, acc.x);
+        acc.y = fmaf(o[s].y, fs, acc.y);
+        acc.z = fmaf(o[s].z, fs, acc.z);
+        acc.w = fmaf(o[s].w, fs, acc.w);
+      }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -481,7 +523,8 @@ __global__ void __launch_bounds__(64)
 // Splits of a row's index list: enough CTAs (two per split, one per value
 // half) to cover the SMs when there are few rows, but at least
 // DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split, since every split costs one
-// query-tile load and one 128 x 512 fp32 partial.
+// query-tile load and one 128 x 512 fp32 partial (one chunk per split doubles
+// the partials' traffic for a 10% faster gather: a net loss).
 static_assert((DSA_MAX_TOPK + kChunk - 1) / kChunk / DSA_MLA_MIN_CHUNKS_PER_SPLIT <= kMaxSplits,
               "the combine holds every split of a row in registers");
 
@@ -523,6 +566,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.ws_o = nullptr;
   p.ws_ml = nullptr;
   p.status = a.status;
+  p.early_inputs = a.early_inputs ? 1 : 0;
   if (ns > 1) {
     p.ws_o = reinterpret_cast<float*>(a.workspace);
     p.ws_ml = p.ws_o + (size_t)n_rows * ns * a.H * kDV;

@@ -406,11 +406,10 @@ struct ClusterSmem {
   uint32_t warp_tot[32];
   uint32_t carry, sel_digit, sel_remaining, n_cand;
   uint32_t above_local, mode, J, aboveJ;
-  uint32_t coarse[64];                 // this CTA's coarse sums (read by every CTA)
+  uint32_t all_coarse[CS][64];         // every CTA's coarse sums (pushed before barrier 1)
   uint32_t tot_coarse[64];             // cluster-wide coarse sums
   uint32_t tot_fine[64];               // cluster-wide fine bins of the chosen coarse bin
   uint32_t g_cnt[CS], g_above[CS];     // from every CTA: candidate count, keys above d*
-  uint32_t g_off[CS + 1];              // exclusive prefix of g_cnt
   uint32_t c_gt[CS], c_eq[CS];         // per source: candidates above / equal to tau
   uint32_t hist[kBins12];              // 12-bit histogram of this slice, later scratch
   uint32_t bitmap[C::kSliceWords];
@@ -496,6 +495,7 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   const int s_lo = min(rank * S, L), s_hi = min(s_lo + S, L);
   const int n = s_hi - s_lo;
   const int n_words = (n + 31) >> 5;
+  cluster_arrive_relaxed();  // "started"; waited for before the first remote store
 
   // ---- 1: keys and 12-bit histogram of the slice, coarse sums
   for (int i = threadIdx.x; i < kBins12; i += NT) sm.hist[i] = 0;
@@ -532,18 +532,24 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
-    if ((threadIdx.x & 7) == 0) sm.coarse[threadIdx.x >> 3] = v;
+    // every lane of the 8-lane group now holds coarse sum c = tid/8; the
+    // group pushes it to all CTAs, lane i of the group to CTAs i, i+8, ...
+    const uint32_t c = threadIdx.x >> 3;
+    cluster_wait();
+#pragma unroll
+    for (int i = 0; i < (CS + 7) / 8; ++i) {
+      const int q = (lane & 7) + 8 * i;
+      if (q < CS) cluster.map_shared_rank(&sm, q)->all_coarse[rank][c] = v;
+    }
   }
-  cluster.sync();  // 1: every histogram and coarse sum is complete
+  cluster.sync();  // 1: every histogram is complete and every coarse sum delivered
 
   // ---- 2: bin d* from the cluster-wide histogram (the same in every CTA).
-  // Entry e = j * CS + q: bin j of CTA q; the CS lanes of a group sum over q.
-  for (int e = threadIdx.x; e < 64 * CS; e += NT) {
-    const int j = e / CS, q = e % CS;
-    uint32_t v = cluster.map_shared_rank(sm.coarse, q)[j];
+  if (threadIdx.x < 64) {
+    uint32_t v = 0;
 #pragma unroll
-    for (int o = CS / 2; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (q == 0) sm.tot_coarse[j] = v;
+    for (int q = 0; q < CS; ++q) v += sm.all_coarse[q][threadIdx.x];
+    sm.tot_coarse[threadIdx.x] = v;
   }
   __syncthreads();
   if (warp == 0) {
@@ -557,12 +563,23 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   }
   __syncthreads();
   const uint32_t J = sm.J, aboveJ = sm.aboveJ;
-  for (int e = threadIdx.x; e < 64 * CS; e += NT) {
-    const int j = e / CS, q = e % CS;
-    uint32_t v = cluster.map_shared_rank(sm.hist, q)[64 * J + j];
+  {  // the 64 fine bins of coarse bin J from every CTA: entry e = j * CS + q;
+     // a thread issues all its remote loads before it uses any
+    constexpr int PER = (64 * CS + NT - 1) / NT;
+    uint32_t v[PER];
 #pragma unroll
-    for (int o = CS / 2; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (q == 0) sm.tot_fine[j] = v;
+    for (int i = 0; i < PER; ++i) {
+      const int e = threadIdx.x + i * NT;
+      v[i] = e < 64 * CS ? cluster.map_shared_rank(sm.hist, e % CS)[64 * J + e / CS] : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = threadIdx.x + i * NT;
+      uint32_t x = v[i];
+#pragma unroll
+      for (int o = CS / 2; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (e < 64 * CS && e % CS == 0) sm.tot_fine[e / CS] = x;
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -614,11 +631,10 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
     __syncthreads();
     const uint32_t nc = sm.n_cand;
     const bool fits = nc <= kPerSrc;
-    if (fits && nc > 0) {
-      for (uint32_t e = threadIdx.x; e < nc * CS; e += NT) {
-        const uint32_t q = e / nc, c = e - q * nc;
-        cluster.map_shared_rank(&sm, (int)q)->g_key[rank][c] = sm.cand_key[c];
-      }
+    if (fits) {  // warp w sends to CTA w % CS, the warps of a destination splitting the list
+      constexpr int WPD = Cfg::kWarps / CS;
+      uint32_t* dst = cluster.map_shared_rank(&sm, warp % CS)->g_key[rank];
+      for (uint32_t c = lane + 32 * (warp / CS); c < nc; c += 32 * WPD) dst[c] = sm.cand_key[c];
     }
     if (threadIdx.x < CS) {
       ClusterSmem<CS>* dst = cluster.map_shared_rank(&sm, (int)threadIdx.x);
@@ -629,34 +645,26 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
   cluster.sync();  // 2: no remote shared-memory access after this point
 
   // ---- 4: exact threshold tau over every candidate, this CTA's offsets, output
-  if (threadIdx.x == 0) {
-    uint32_t tot = 0, bad = 0;
-    for (int q = 0; q < CS; ++q) {
-      sm.g_off[q] = tot;
-      if (sm.g_cnt[q] == 0xFFFFFFFFu) bad = 1;
-      else tot += sm.g_cnt[q];
+  {
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < CS; ++q) bad |= sm.g_cnt[q] == 0xFFFFFFFFu;
+    if (bad) {  // a CTA had too many keys in bin d*: rank 0 redoes the row alone
+      if (rank == 0) radix_select_fallback<NT>(sm, sm.keys, Cfg::kSliceMax, row, L, k, out);
+      return;
     }
-    sm.g_off[CS] = tot;
-    sm.mode = bad;
   }
-  __syncthreads();
-  if (sm.mode) {  // a CTA had too many keys in bin d*: rank 0 redoes the row alone
-    if (rank == 0) radix_select_fallback<NT>(sm, sm.keys, Cfg::kSliceMax, row, L, k, out);
-    return;
-  }
-  const uint32_t n_all = sm.g_off[CS];
+  constexpr int WPS = Cfg::kWarps / CS;  // warps per source CTA
+  const int src = warp % CS;
+  const uint32_t src_cnt = sm.g_cnt[src];
   uint32_t prefix = dstar << 20, pmask = 0xFFF00000u, remaining = need_in_bin;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? 10 : 0;
     for (int i = threadIdx.x; i < 1024; i += NT) sm.hist[i] = 0;
     __syncthreads();
-    for (uint32_t c = threadIdx.x; c < n_all; c += NT) {
-      int q = 0;  // source of dense index c: the last q with g_off[q] <= c
-#pragma unroll
-      for (int step = CS / 2; step; step >>= 1)
-        if (q + step < CS && sm.g_off[q + step] <= c) q += step;
-      const uint32_t key = sm.g_key[q][c - sm.g_off[q]];
+    for (uint32_t c = lane + 32 * (warp / CS); c < src_cnt; c += 32 * WPS) {
+      const uint32_t key = sm.g_key[src][c];
       if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
     }
     __syncthreads();
@@ -667,11 +675,15 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
     __syncthreads();
   }
   const uint32_t tau = prefix, need_eq = remaining;
-  if (warp < CS) {  // per source: candidates above and equal to tau
-    const uint32_t cnt = sm.g_cnt[warp];
+  if (threadIdx.x < CS) {
+    sm.c_gt[threadIdx.x] = 0;
+    sm.c_eq[threadIdx.x] = 0;
+  }
+  __syncthreads();
+  {  // per source: candidates above and equal to tau
     uint32_t gt = 0, eq = 0;
-    for (uint32_t i = lane; i < cnt; i += 32) {
-      const uint32_t key = sm.g_key[warp][i];
+    for (uint32_t c = lane + 32 * (warp / CS); c < src_cnt; c += 32 * WPS) {
+      const uint32_t key = sm.g_key[src][c];
       gt += key > tau;
       eq += key == tau;
     }
@@ -680,9 +692,9 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
       gt += __shfl_xor_sync(0xffffffffu, gt, o);
       eq += __shfl_xor_sync(0xffffffffu, eq, o);
     }
-    if (lane == 0) {
-      sm.c_gt[warp] = gt;
-      sm.c_eq[warp] = eq;
+    if (lane == 0 && (gt | eq)) {
+      atomicAdd(&sm.c_gt[src], gt);
+      atomicAdd(&sm.c_eq[src], eq);
     }
   }
   __syncthreads();
@@ -698,26 +710,26 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
     else if (key == tau) atomicOr(&sm.eqmap[s >> 5], 1u << (s & 31));
   }
   __syncthreads();
-  {  // keys equal to tau: keep those whose rank over the whole row is below need_eq
+  {  // one scan gives, per bitmap word, the kept keys above tau and the keys
+     // equal to tau before it; equal keys are kept in position order while
+     // their rank over the whole row is below need_eq
     const int w = threadIdx.x;
-    uint32_t bits = w < Cfg::kSliceWords ? sm.eqmap[w] : 0u;
+    const uint32_t up = w < Cfg::kSliceWords ? sm.bitmap[w] : 0u;
+    uint32_t eqb = w < Cfg::kSliceWords ? sm.eqmap[w] : 0u;
     uint32_t tot;
-    uint32_t rk = eq_base + block_excl_scan<NT>((uint32_t)__popc(bits), sm, &tot);
+    const uint32_t packed = block_excl_scan<NT>((uint32_t)__popc(up) | ((uint32_t)__popc(eqb) << 16), sm, &tot);
+    uint32_t rk = eq_base + (packed >> 16);  // rank of this word's first equal key
+    const uint32_t quota = need_eq > eq_base ? need_eq - eq_base : 0u;
+    const uint32_t eq_kept_before = min(packed >> 16, quota);
     uint32_t keep = 0;
-    while (bits && rk < need_eq) {
-      const uint32_t low = bits & (0u - bits);
+    while (eqb && rk < need_eq) {
+      const uint32_t low = eqb & (0u - eqb);
       keep |= low;
-      bits ^= low;
+      eqb ^= low;
       ++rk;
     }
-    if (keep) sm.bitmap[w] |= keep;
-  }
-  __syncthreads();
-  {  // ascending output of this slice at its offset: one bitmap word per thread
-    const int w = threadIdx.x;
-    uint32_t bits = w < Cfg::kSliceWords ? sm.bitmap[w] : 0u;
-    uint32_t tot;
-    uint32_t pos = out_base + block_excl_scan<NT>((uint32_t)__popc(bits), sm, &tot);
+    uint32_t bits = up | keep;
+    uint32_t pos = out_base + (packed & 0xFFFFu) + eq_kept_before;
     while (bits) {
       const int bb = __ffs(bits) - 1;
       bits &= bits - 1;
