@@ -140,7 +140,7 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
  * allocator, a serving loop whose memory is fixed at start-up, code that may
  * not call cudaMalloc on that path).  Same arguments, layouts and results as
  * dsa_sparse_mla, minus the workspace: the split partials live in a scratch
- * array of DSA_NOALLOC_SCRATCH_BYTES (64 MiB) built into the library, which
+ * array of DSA_NOALLOC_SCRATCH_BYTES (32 MiB) built into the library, which
  * every GPU that loads the library holds until the process exits.
  *   - A call that needs more scratch than that (dsa_sparse_mla_workspace_size
  *     above the limit; e.g. 128..147 rows at H = 128, k = 2048) returns
@@ -154,7 +154,7 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
  *   - Nothing in the scratch needs to start at zero: every value a call reads
  *     was written earlier in the same call.
  */
-#define DSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+#define DSA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 int dsa_sparse_mla_noalloc(const void* q, const void* kv, const int32_t* offsets,
                            const int32_t* indices, int B, int T, int H, int k, float scale,
                            int64_t kv_rows, void* out, int out_dtype, float* lse,

@@ -9,7 +9,7 @@
 // entry point keeps the split partials of the sparse-MLA stage in a fixed
 // scratch array that is part of the library image itself.
 //
-// The scratch is a file-scope device array of kScratchBytes (64 MiB).  Every
+// The scratch is a file-scope device array of kScratchBytes (32 MiB).  Every
 // GPU that loads the library holds it until the process exits.  Its device
 // address is looked up once per device with cudaGetSymbolAddress (the host
 // side name of the array is only a stand-in, not a device address).
@@ -21,7 +21,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = DSA_NOALLOC_SCRATCH_BYTES;
-static_assert(kScratchBytes == (64ull << 20), "the header states 64 MiB");
+static_assert(kScratchBytes == (32ull << 20), "the header states 32 MiB");
 
 static __device__ __align__(256) unsigned char g_mla_scratch[kScratchBytes];
 

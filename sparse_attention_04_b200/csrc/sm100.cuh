@@ -121,6 +121,15 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // its shared-memory source (the global writes complete by kernel end).
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// 2-D tiled bulk tensor store shared -> global (bulk-group completion).  The
+// shared-memory box is laid out as the tensor map's swizzle describes.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 
 // 16-byte async copy; src_bytes = 0 writes zeros (nothing is read).

@@ -17,7 +17,7 @@
 // The running max m is only raised when a chunk exceeds it by more than
 // 2^8 (then O and the running sum are rescaled), so P <= 256 and the
 // final O / l is exact softmax.  With more than one split, the unnormalised
-// O and (m, l) go to the workspace and dsa_mla_combine merges them.
+// O (bf16) and (m, l) go to the workspace and the combine kernel merges them.
 //
 // TMEM: O half in columns [0,256), S in two 32-column buffers at 256 and 288.
 // Shared memory: Q (128 x 576 bf16, 9 swizzled 64-column blocks, by TMA), two
@@ -48,8 +48,8 @@ constexpr int kOffP = kOffKv + 2 * kKvBytes;
 constexpr int kOffBar = kOffP + kPBytes;
 constexpr int kNumBar = 9;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
-constexpr int kStageRow = 1040;                  // epilogue staging: 1 KiB + 16 per head
-static_assert(128 * kStageRow <= kQBytes, "the staged output fits where the query tile was");
+constexpr int kStageBlock = 128 * 128;           // epilogue staging: one box, 128 rows x 128 B
+static_assert(8 * kStageBlock <= kQBytes, "the staged output fits where the query tile was");
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
@@ -73,8 +73,8 @@ struct MlaParams {
   void* out;
   int out_bf16;
   float* lse;
-  float* ws_o;   // [rows][splits][H][512]   (n_splits > 1)
-  float* ws_ml;  // [rows][splits][H][2]
+  __nv_bfloat16* ws_o;  // [rows][splits][H][512] unnormalised partials (n_splits > 1)
+  float* ws_ml;          // [rows][splits][H][2]   their (max, sum)
   int32_t* status;
   int early_inputs;  // q and offsets may be read before the dependency wait
 };
@@ -82,7 +82,8 @@ struct MlaParams {
 __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 && idx < E; }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
+                      const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -175,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (v == 0 && p.lse) p.lse[rh] = -INFINITY;
       } else {
         const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
-        float* o = p.ws_o + slot * kDV + 256 * v;
-        for (int c = 0; c < 256; ++c) o[c] = 0.f;
+        __nv_bfloat16* o = p.ws_o + slot * kDV + 256 * v;
+        for (int c = 0; c < 256; ++c) o[c] = __float2bfloat16(0.f);
         if (v == 0) {
           p.ws_ml[2 * slot] = -INFINITY;
           p.ws_ml[2 * slot + 1] = 0.f;
@@ -344,17 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(p_full);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_my - 1) & 1, abort, kWaitLimitNs));
+    // Every MMA has completed, so the query tile's shared memory is free: the
+    // 128 x 256 result is staged there as 128-byte-swizzled boxes of 32 fp32
+    // (or 64 bf16) columns, one thread per head row, and written by a few
+    // TMA tensor stores (the output's tensor map has one box per such block).
+    const bool final_out = p.n_splits == 1;
+    const bool as_bf16 = !final_out || p.out_bf16;  // partials are bf16 too
     if (ok) {
-      // Every MMA has completed, so the query tile's shared memory is free:
-      // each thread stages its head's 256 values there (rows 1040 bytes
-      // apart, conflict-free) and writes them with one bulk copy.
       tc_fence_after();
-      const int64_t rh = (int64_t)r * p.H + h;
-      const bool write = h < p.H;
-      const bool final_out = p.n_splits == 1;
-      const bool as_bf16 = final_out && p.out_bf16;
       const float mul = final_out ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
-      uint8_t* srow = smem + kOffQ + h * kStageRow;
+      uint8_t* stage = smem + kOffQ;
+      const int sw = h & 7;
 #pragma unroll 1
       for (int cb2 = 0; cb2 < 8; cb2 += 2) {
         uint32_t ovp[2][32];
@@ -362,54 +363,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_addr + 32 * cb2 + 32, ovp[1]);
         tc_wait_ld();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-        const int cb = cb2 + half;
-        const uint32_t (&ov)[32] = ovp[half];
-        if (as_bf16) {
-          uint4* d = reinterpret_cast<uint4*>(srow + cb * 64);
+        for (int hf = 0; hf < 2; ++hf) {
+          const int cb = cb2 + hf;
+          const uint32_t (&ov)[32] = ovp[hf];
+          if (as_bf16) {
+            uint8_t* rowp = stage + (cb >> 1) * kStageBlock + h * 128;
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w4[4];
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t w4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q4 + 2 * e]) * mul,
-                                                               __uint_as_float(ov[8 * q4 + 2 * e + 1]) * mul);
-              w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q4 + 2 * e]) * mul,
+                                                                 __uint_as_float(ov[8 * q4 + 2 * e + 1]) * mul);
+                w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
+              }
+              const int ci = (cb & 1) * 4 + q4;
+              *reinterpret_cast<uint4*>(rowp + ((ci ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            d[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        } else {
-          float4* d = reinterpret_cast<float4*>(srow + cb * 128);
+          } else {
+            uint8_t* rowp = stage + cb * kStageBlock + h * 128;
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            d[q4] = make_float4(__uint_as_float(ov[4 * q4]) * mul, __uint_as_float(ov[4 * q4 + 1]) * mul,
-                                __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
-        }
-        }
-      }
-      if (write) {
-        fence_proxy_async_smem();
-        void* dst;
-        if (!final_out)
-          dst = p.ws_o + (((int64_t)r * p.n_splits + sp) * p.H + h) * kDV + 256 * v;
-        else if (p.out_bf16)
-          dst = reinterpret_cast<__nv_bfloat16*>(p.out) + rh * kDV + 256 * v;
-        else
-          dst = reinterpret_cast<float*>(p.out) + rh * kDV + 256 * v;
-        bulk_store_s2g(dst, smem_u32(srow), as_bf16 ? 512u : 1024u);
-        bulk_commit();
-      }
-      if (write && v == 0) {
-        if (final_out) {
-          if (p.lse) p.lse[rh] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-        } else {
-          const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
-          p.ws_ml[2 * slot] = l_run > 0.f ? m_run : -INFINITY;
-          p.ws_ml[2 * slot + 1] = l_run;
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(rowp + ((q4 ^ sw) << 4)) =
+                  make_float4(__uint_as_float(ov[4 * q4]) * mul, __uint_as_float(ov[4 * q4 + 1]) * mul,
+                              __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
+          }
         }
       }
-      if (write) bulk_wait_read();  // shared memory stays valid until the copy has read it
+      fence_proxy_async_smem();
     }
+    named_barrier_sync(1, 128);  // every epilogue warp, whatever its wait outcome
+    if (threadIdx.x == 0 && !*abort) {
+      const int nblk = as_bf16 ? 4 : 8, colw = as_bf16 ? 64 : 32;
+      const int y = final_out ? r * p.H : (r * p.n_splits + sp) * p.H;
+      for (int bk = 0; bk < nblk; ++bk) tma_store_2d(&tm_out, sbase + kOffQ + bk * kStageBlock, 256 * v + colw * bk, y);
+      bulk_commit();
+    }
+    if (ok && h < p.H && v == 0) {
+      const int64_t rh = (int64_t)r * p.H + h;
+      if (final_out) {
+        if (p.lse) p.lse[rh] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      } else {
+        const int64_t slot = ((int64_t)r * p.n_splits + sp) * p.H + h;
+        p.ws_ml[2 * slot] = l_run > 0.f ? m_run : -INFINITY;
+        p.ws_ml[2 * slot + 1] = l_run;
+      }
+    }
+    if (threadIdx.x == 0) bulk_wait_read();  // the staged boxes stay valid until read
   }
 
   tc_fence_before();
@@ -423,27 +423,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
-// Two CTAs of 64 threads per (row, head), one per column half; thread c owns
-// four columns and issues the loads of every split at once.
+// One CTA of 64 threads per (row, head); thread c owns eight columns and
+// issues the 16-byte loads of 32 splits at once.
 constexpr int kMaxSplits = 64;
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+    acc[2 * e] = fmaf(t.x, f, acc[2 * e]);
+    acc[2 * e + 1] = fmaf(t.y, f, acc[2 * e + 1]);
+  }
+}
+
 __global__ void __launch_bounds__(64)
-    mla_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
+    mla_combine_kernel(const __nv_bfloat16* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
   __shared__ float s_w[kMaxSplits];
   __shared__ float s_ml[2];
   grid_dependency_wait();  // partials come from the previous kernel
   allow_dependents_launch();
-  const int64_t rh = blockIdx.x >> 1;  // row * H + head
-  const int half = blockIdx.x & 1;
+  const int64_t rh = blockIdx.x;  // row * H + head
   const int64_t r = rh / H, h = rh % H;
-  const int c4 = half * 64 + threadIdx.x;  // float4 column of the 512
-  const float4* base = reinterpret_cast<const float4*>(ws_o + (r * n_splits * H + h) * kDV) + c4;
-  const int64_t stride4 = (int64_t)H * kDV / 4;  // between consecutive splits
-  // the first 32 splits' loads are issued before the weights are known
-  float4 o[32];
+  const int c8 = threadIdx.x;  // eight columns: 8*c8 .. 8*c8+7
+  const uint4* base = reinterpret_cast<const uint4*>(ws_o + (r * n_splits * H + h) * kDV) + c8;
+  const int64_t stride = (int64_t)H * kDV / 8;  // uint4 between consecutive splits
+  uint4 o[32];
 #pragma unroll
   for (int s = 0; s < 32; ++s)
-    if (s < n_splits) o[s] = __ldg(base + s * stride4);
+    if (s < n_splits) o[s] = __ldg(base + s * stride);
   if (threadIdx.x < 32) {
     const int s0 = threadIdx.x, s1 = threadIdx.x + 32;
     float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
@@ -474,44 +482,34 @@ __global__ void __launch_bounds__(64)
   }
   __syncthreads();
   const float M = s_ml[0], L = s_ml[1];
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int s = 0; s < 32; ++s) {
-    if (s < n_splits) {
-      const float fs = s_w[s];
-      acc.x = fmaf(o[s].x, fs, acc.x);
-      acc.y = fmaf(o[s].y, fs, acc.y);
-      acc.z = fmaf(o[s].z, fs, acc.z);
-      acc.w = fmaf(o[s].w, fs, acc.w);
-    }
-  }
+  for (int s = 0; s < 32; ++s)
+    if (s < n_splits) acc_bf16x8(acc, o[s], s_w[s]);
   if (n_splits > 32) {  // the second group of splits
 #pragma unroll
     for (int s = 0; s < 32; ++s)
-      if (32 + s < n_splits) o[s] = __ldg(base + (32 + s) * stride4);
+      if (32 + s < n_splits) o[s] = __ldg(base + (32 + s) * stride);
 #pragma unroll
-    for (int s = 0; s < 32; ++s) {
-      if (32 + s < n_splits) {
-        const float fs = s_w[32 + s];
-        acc.x = fmaf(o[s].x, fs, acc.x);
-        acc.y = fmaf(o[s].y, fs, acc.y);
-        acc.z = fmaf(o[s].z, fs, acc.z);
-        acc.w = fmaf(o[s].w, fs, acc.w);
-      }
-    }
+    for (int s = 0; s < 32; ++s)
+      if (32 + s < n_splits) acc_bf16x8(acc, o[s], s_w[32 + s]);
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if (out_bf16) {
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + rh * kDV)[c4] =
-        make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 t2 = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+      w4[e] = *reinterpret_cast<const uint32_t*>(&t2);
+    }
+    reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + rh * kDV)[c8] =
+        make_uint4(w4[0], w4[1], w4[2], w4[3]);
   } else {
-    reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + rh * kDV)[c4] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    float4* o4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + rh * kDV) + 2 * c8;
+    o4[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    o4[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
   }
-  if (half == 0 && threadIdx.x == 0 && lse)
-    lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  if (threadIdx.x == 0 && lse) lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace
@@ -523,8 +521,8 @@ __global__ void __launch_bounds__(64)
 // Splits of a row's index list: enough CTAs (two per split, one per value
 // half) to cover the SMs when there are few rows, but at least
 // DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split, since every split costs one
-// query-tile load and one 128 x 512 fp32 partial (one chunk per split doubles
-// the partials' traffic for a 10% faster gather: a net loss).
+// query-tile load and one 128 x 512 partial (one chunk per split doubles the
+// partials' traffic for a 10% faster gather: a net loss).
 static_assert((DSA_MAX_TOPK + kChunk - 1) / kChunk / DSA_MLA_MIN_CHUNKS_PER_SPLIT <= kMaxSplits,
               "the combine holds every split of a row in registers");
 
@@ -542,7 +540,7 @@ int mla_num_splits(int n_rows, int k) {
 size_t mla_workspace_bytes(int n_rows, int H, int k) {
   const int ns = mla_num_splits(n_rows, k);
   if (ns <= 1) return 0;
-  return (size_t)n_rows * ns * H * (kDV + 2) * sizeof(float);
+  return (size_t)n_rows * ns * H * (kDV * sizeof(__nv_bfloat16) + 2 * sizeof(float));
 }
 
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
@@ -568,13 +566,25 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
   if (ns > 1) {
-    p.ws_o = reinterpret_cast<float*>(a.workspace);
-    p.ws_ml = p.ws_o + (size_t)n_rows * ns * a.H * kDV;
+    p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);
+    p.ws_ml = reinterpret_cast<float*>(p.ws_o + (size_t)n_rows * ns * a.H * kDV);
   }
-  CUtensorMap tq;
+  CUtensorMap tq, tout;
   if (!make_tmap_2d(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)n_rows * a.H,
                     kDQK * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
+  // where the epilogue's boxes go: the split partials (bf16), or the output
+  bool tm_ok;
+  if (ns > 1)
+    tm_ok = make_tmap_2d(&tout, p.ws_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDV, (uint64_t)n_rows * ns * a.H,
+                         kDV * 2, 64, (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
+  else if (p.out_bf16)
+    tm_ok = make_tmap_2d(&tout, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDV, (uint64_t)n_rows * a.H, kDV * 2, 64,
+                         (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    tm_ok = make_tmap_2d(&tout, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDV, (uint64_t)n_rows * a.H, kDV * 4, 32,
+                         (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!tm_ok) return DSA_ERR_CUDA;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -583,12 +593,12 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   const int64_t grid = (int64_t)n_rows * ns * 2;
-  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, p) !=
+  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (ns > 1) {
-    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H * 2)), dim3(64), 0, stream,
-                   (const float*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=
+    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(64), 0, stream,
+                   (const __nv_bfloat16*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
   }

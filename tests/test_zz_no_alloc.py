@@ -56,8 +56,8 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device, B, E):
 
 def test_noalloc_rejects_work_beyond_its_scratch(cuda_device):
     from sparse_attention_04_b200 import _lib
-    # a row count whose split partials exceed the built-in 64 MiB
-    limit = 64 << 20
+    # a row count whose split partials exceed the built-in 32 MiB
+    limit = 32 << 20
     rows = next(r for r in range(1, 4096) if _lib.sparse_mla_workspace_size(r, 1, 128, 2048) > limit)
     dummy = torch.zeros(16, dtype=torch.uint8, device=cuda_device)
     rc = _lib.lib.dsa_sparse_mla_noalloc(_lib._p(dummy), _lib._p(dummy), _lib._p(dummy), _lib._p(dummy), rows, 1,
