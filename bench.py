@@ -76,28 +76,78 @@ def oracle_work(wl, end_pos):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock, its maximum and the clock-event (throttle) reasons of one GPU,
+    sampled every few milliseconds on a background thread through NVML while
+    the timed region runs; falls back to `nvidia-smi -lms` when NVML is
+    unavailable."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, device, period_s=0.005):
+        self.device = device
+        self.period = period_s
+        self.samples = []      # (sm_mhz, max_mhz, reasons_mask)
+        self.thread = None
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+        self.stop_flag = False
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
 
     def start(self):
+        import threading
         try:
+            import pynvml
+            h = self._nvml_handle()
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+
+            def loop():
+                while not self.stop_flag:
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                             int(get_reasons(h))))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
+        try:  # fallback: nvidia-smi polling
+            self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.device.index or 0), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+            sm = [x[0] for x in self.samples]
+            reasons = sorted({name for _, _, m in self.samples for bit, name in self.REASONS.items() if m & bit})
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": self.samples[0][1] if self.samples else None,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml"}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -118,7 +168,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -271,16 +321,16 @@ def run_native(args, rank, world, local):
     launches_per_step = 3 + (1 if _lib.sparse_mla_workspace_size(wl.B, 1, wl.H, wl.topk) > 0 else 0)
 
     # ---- warm-up (untimed)
-    clocks = ClockSampler(local)
-    clocks.start()
     for _ in range(max(1, W // max(1, min(W, G)))):
         if graph_warm is not None:
             graph_warm.replay()
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly K steps
+    # ---- timed region: exactly K steps (clocks sampled throughout)
     if world > 1:
         torch.distributed.barrier()
+    clocks = ClockSampler(dev)
+    clocks.start()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -511,7 +561,7 @@ def run_prefill_only(args, rank, world, dev):
     except Exception:
         peaks = {}
     stream = torch.cuda.Stream(dev)
-    clocks = ClockSampler(dev.index or 0)
+    clocks = ClockSampler(dev)
     clocks.start()
     res = run_prefill(dev, stream, peaks, reps=max(1, args.steps))
     clk = clocks.stop()
