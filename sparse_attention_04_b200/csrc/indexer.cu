@@ -61,7 +61,13 @@ struct IdxCfg {
   static constexpr int OFF_BAR = OFF_W + 2 * N * 4;
   static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  // The swizzled tiles need 1 KiB alignment.  Where the budget allows, 1 KiB
+  // of slack lets the kernel align the base itself; otherwise (the bf16
+  // prefill ring) it relies on the dynamic shared memory base being 1 KiB
+  // aligned and reports DSA_ERR_UNSUPPORTED, without touching memory, if not.
+  static constexpr int USED_BYTES = OFF_MISC + 64;
+  static constexpr bool SLACK = USED_BYTES + 1024 <= 232448;
+  static constexpr int SMEM_BYTES = USED_BYTES + (SLACK ? 1024 : 0);
   static constexpr int THREADS = 32 * (EPI_WARPS + 2);
   static_assert(NQ % (EPI_WARPS / 4) == 0, "queries split evenly over the warps of a lane quarter");
   static_assert(N <= 256, "MMA N limit");
@@ -173,6 +179,10 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
                    float* __restrict__ scores, int64_t ld, int32_t* status) {
   using C = IdxCfg<NQ, FP8>;
   extern __shared__ uint8_t smem_raw[];
+  if (!C::SLACK && (smem_u32(smem_raw) & 1023u) != 0) {  // uniform over the CTA
+    if (threadIdx.x == 0) report(status, DSA_ERR_UNSUPPORTED);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
@@ -388,24 +398,28 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
       const int s = kt * 128 + row;
       float ksc = 1.f;
       if (FP8 && s < E) ksc = k_scale[base_row + s];
-#pragma unroll 1
+      // every TMEM load of the warp's queries first, then one wait
+      uint32_t v[C::QPW][2][32];
+#pragma unroll
+      for (int qq = 0; qq < C::QPW; ++qq) {
+        tmem_ld32(lane_addr + ab * C::N + (q_lo + qq) * 64, v[qq][0]);
+        tmem_ld32(lane_addr + ab * C::N + (q_lo + qq) * 64 + 32, v[qq][1]);
+      }
+      tc_wait_ld();
+      // the accumulator is in registers: hand its TMEM buffer back to the MMA now
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(ab));
+#pragma unroll
       for (int qq = 0; qq < C::QPW; ++qq) {
         const int q = q_lo + qq;
-        uint32_t v0[32], v1[32];
-        tmem_ld32(lane_addr + ab * C::N + q * 64, v0);
-        tmem_ld32(lane_addr + ab * C::N + q * 64 + 32, v1);
-        tc_wait_ld();
-        const float score = head_sum64(v0, v1, w_s + (qord & 1) * C::N + q * 64) * ksc;
+        const float score = head_sum64(v[qq][0], v[qq][1], w_s + (qord & 1) * C::N + q * 64) * ksc;
         const int t = qb * NQ + q;
         if (t < T && s < E)
           scores[((int64_t)b * T + t) * ld + s] = (s <= start + t) ? score : -INFINITY;
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(acc_empty(ab));
-        if (kt + 1 == len || item + 1 == count) mbar_arrive(q_empty(qord & 1));  // block done
-      }
+      if (lane == 0 && (kt + 1 == len || item + 1 == count)) mbar_arrive(q_empty(qord & 1));  // block done
       if (++kt == len && item + 1 < count) {
         ++seg;
         kt = 0;
