@@ -78,6 +78,7 @@ struct MlaArgs {
 };
 int mla_num_splits(int n_rows, int k);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
+bool mla_pregather(int n_rows, int k);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
 
 // Launches `kernel` on `stream` with programmatic stream serialisation, so

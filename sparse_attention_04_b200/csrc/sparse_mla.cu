@@ -30,6 +30,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "dsa_internal.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -50,7 +52,8 @@ constexpr int kNumBar = 9;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
 constexpr int kStageBlock = 128 * 128;           // epilogue staging: one box, 128 rows x 128 B
 static_assert(8 * kStageBlock <= kQBytes, "the staged output fits where the query tile was");
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kMiscBytes = 64 + 4 * ((DSA_MAX_TOPK + kChunk - 1) / kChunk);  // MlaMisc
+constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kIdescQK = idesc_bf16(128, kChunk);
@@ -58,9 +61,12 @@ constexpr uint32_t kIdescPV = idesc_bf16(128, 256, /*b_mn_major=*/true);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffKv % 1024 == 0 && kOffP % 1024 == 0, "alignment");
 
+constexpr int kMaxChunks = (DSA_MAX_TOPK + kChunk - 1) / kChunk;
 struct MlaMisc {
   int tmem_base, abort, n_chunks, last_valid, pad[12];
+  uint32_t vmask[kMaxChunks];  // per chunk of this split: bit j = position valid
 };
+static_assert(sizeof(MlaMisc) == kMiscBytes, "shared-memory budget of the bookkeeping block");
 
 struct MlaParams {
   const __nv_bfloat16* kv;
@@ -77,13 +83,14 @@ struct MlaParams {
   float* ws_ml;          // [rows][splits][H][2]   their (max, sum)
   int32_t* status;
   int early_inputs;  // q and offsets may be read before the dependency wait
+  int pregathered;   // rows already copied into a dense buffer: TMA tile loads
 };
 
 __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 && idx < E; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                      const MlaParams p) {
+                      const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -117,11 +124,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     misc->last_valid = -1;
     misc->abort = 0;
   }
+  if (threadIdx.x < kMaxChunks) misc->vmask[threadIdx.x] = 0u;
   if (warp == 8) {
     if (lane == 0) {
       mbar_init(q_full, 1);
       for (int i = 0; i < 2; ++i) {
-        mbar_init(kv_full(i), 64);  // the gather group of that stage
+        mbar_init(kv_full(i), p.pregathered ? 1 : 64);  // TMA expect-tx, or the gather group
         mbar_init(kv_empty(i), 1);
         mbar_init(s_full(i), 1);
       }
@@ -150,8 +158,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lv = -1;
     for (int j = c_begin * kChunk + threadIdx.x; j < min(c_end * kChunk, p.k); j += kThreads) {
       const int32_t id = idx_row[j];
-      if (index_ok(id, E)) lv = j;
-      else if (id != -1) report(p.status, DSA_ERR_BAD_INDEX);
+      if (index_ok(id, E)) {
+        lv = j;
+        atomicOr(&misc->vmask[j / kChunk - c_begin], 1u << (j % kChunk));
+      } else if (id != -1) {
+        report(p.status, DSA_ERR_BAD_INDEX);
+      }
     }
     if (lv >= 0) atomicMax(&misc->last_valid, lv);
   } else if (threadIdx.x == 0) {
@@ -190,11 +202,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 8) {
     // -------------------------------------------------------------- MMA issuer
+    // QK of chunk i and PV of chunk j < i touch different TMEM (S buffer,
+    // O) and shared memory (stage i; stage j and P), so they are issued in
+    // whichever order their inputs arrive: QK(i) once chunk i has landed and
+    // its S buffer is free (PV(i-2) issued, so softmax(i-2) is done with it);
+    // PV(j) once softmax(j) has written P.  An early PV(j) frees its stage for
+    // the load of chunk j+2 without waiting for chunk j+1 to land.
     if (lane == 0) {
-      int done_pv = 0;
+      int n_qk = 0, n_pv = 0;
       bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(p_full, j & 1, abort, kWaitLimitNs)) return false;
+      // PV of chunk n_pv (its P is in shared memory; p_full has been seen)
+      auto issue_pv = [&]() {
+        const int j = n_pv;
         tc_fence_after();
         const uint32_t kvb = sbase + kOffKv + (j & 1) * kKvBytes + (4 * v) * (kChunk * 128);
 #pragma unroll
@@ -205,30 +224,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(pv_done);
         tc_commit(kv_empty(j & 1));
-        done_pv = j + 1;
-        return true;
+        ++n_pv;
       };
-      for (int i = 0; ok && i < n_my; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(kv_full(st), (i >> 1) & 1, abort, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kvb = sbase + kOffKv + st * kKvBytes;
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t spins = 0;
+      while (ok && n_pv < n_my) {
+        bool progressed = false;
+        if (n_qk < n_my && n_qk <= n_pv + 1 && mbar_try_wait(kv_full(n_qk & 1), (n_qk >> 1) & 1)) {
+          const int st = n_qk & 1;
+          tc_fence_after();
+          const uint32_t kvb = sbase + kOffKv + st * kKvBytes;
 #pragma unroll 1
-        for (int kb = 0; kb < kKB; ++kb) {
+          for (int kb = 0; kb < kKB; ++kb) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc(sbase + kOffQ + kb * 16384 + ks * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(kvb + kb * (kChunk * 128) + ks * 32, 16, 1024, kSwizzle128B);
-            mma_f16_ss(tmem + 256 + 32 * st, ad, bd, kIdescQK, (kb | ks) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc(sbase + kOffQ + kb * 16384 + ks * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(kvb + kb * (kChunk * 128) + ks * 32, 16, 1024, kSwizzle128B);
+              mma_f16_ss(tmem + 256 + 32 * st, ad, bd, kIdescQK, (kb | ks) ? 1u : 0u);
+            }
+            // a PV whose P is ready is slotted in between the groups of QK
+            // MMAs, instead of waiting for the whole (slow, N = 32) QK
+            if (n_pv < n_qk && mbar_try_wait(p_full, n_pv & 1)) issue_pv();
+          }
+          tc_commit(s_full(st));
+          ++n_qk;
+          progressed = true;
+        }
+        if (n_pv < n_qk && mbar_try_wait(p_full, n_pv & 1)) {
+          issue_pv();
+          progressed = true;
+        }
+        if (!progressed && (++spins & 63u) == 0) {  // bounded, like every other wait here
+          if (*abort) ok = false;
+          else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            ok = false;
           }
         }
-        tc_commit(s_full(st));
-        if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(n_my - 1);
-      if (*abort && done_pv > 0) {  // tensor-core work must finish before TMEM is released
+      if (*abort && n_pv > 0) {  // tensor-core work must finish before TMEM is released
         volatile int never = 0;
-        mbar_wait(pv_done, (done_pv - 1) & 1, &never, 10000000ull);
+        mbar_wait(pv_done, (n_pv - 1) & 1, &never, 10000000ull);
       }
       if (*abort) {
         volatile int never = 0;
@@ -237,44 +273,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- row gather
-    // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
-    // the two groups run independently, so both stages are in flight from
-    // the start and a group waits only for its own copies before it signals.
-    // Each warp copies 16 whole rows, one row at a time, so every copy
-    // instruction reads 512 contiguous bytes of a row.
-    const int pt = threadIdx.x - 128;
-    const int grp = pt >> 6, gw = (pt >> 5) & 1;
-    const __nv_bfloat16* kv = p.kv;
-    for (int i = grp; i < n_my; i += 2) {
-      const int st = i & 1;
-      if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
-      int32_t my_id = -1;
-      if (lane < 16) {
-        const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
-        my_id = pos < p.k ? idx_row[pos] : -1;
-      }
-#pragma unroll 2
-      for (int rr = 0; rr < 16; ++rr) {
-        const int jr = gw * 16 + rr;
-        const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
-        const bool valid = index_ok(id, E);
-        const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
-        const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
-#pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
-          if (c < kDQK / 8) {
-            const int kb = c >> 3, cc = c & 7;
-            cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
-          }
+    if (p.pregathered) {
+      // The rows were copied into a dense [rows * k, 576] buffer by the gather
+      // kernel: each chunk is 9 tiled TMA loads of 32 rows x 64 columns,
+      // landing in the same swizzled K-major layout.
+      if (threadIdx.x == 128) {
+        int issued = 0;
+        for (int i = 0; i < n_my; ++i) {
+          const int st = i & 1;
+          if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+          mbar_arrive_expect_tx(kv_full(st), kKvBytes);
+          const int row0 = r * p.k + (c_begin + i) * kChunk;
+          for (int kb = 0; kb < kKB; ++kb)
+            tma_load_2d(sbase + kOffKv + st * kKvBytes + kb * (kChunk * 128), &tm_kv, kb * 64, row0, kv_full(st));
+          issued = i + 1;
+        }
+        if (*abort) {  // let copies in flight land before the CTA exits
+          volatile int never = 0;
+          for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(kv_full(i & 1), (i >> 1) & 1, &never, 10000000ull);
         }
       }
-      cp_async_commit();
+    } else {
+      // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
+      // the two groups run independently, so both stages are in flight from
+      // the start and a group waits only for its own copies before it signals.
+      // Each warp copies 16 whole rows, one row at a time, so every copy
+      // instruction reads 512 contiguous bytes of a row.
+      const int pt = threadIdx.x - 128;
+      const int grp = pt >> 6, gw = (pt >> 5) & 1;
+      const __nv_bfloat16* kv = p.kv;
+      for (int i = grp; i < n_my; i += 2) {
+        const int st = i & 1;
+        if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+        int32_t my_id = -1;
+        if (lane < 16) {
+          const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
+          my_id = pos < p.k ? idx_row[pos] : -1;
+        }
+  #pragma unroll 2
+        for (int rr = 0; rr < 16; ++rr) {
+          const int jr = gw * 16 + rr;
+          const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
+          const bool valid = index_ok(id, E);
+          const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
+          const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
+  #pragma unroll
+          for (int u = 0; u < 3; ++u) {
+            const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
+            if (c < kDQK / 8) {
+              const int kb = c >> 3, cc = c & 7;
+              cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+            }
+          }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(kv_full(st));
+      }
       cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(kv_full(st));
     }
-    cp_async_wait<0>();
   } else {
     // -------------------------------------------------------------- softmax + epilogue
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -290,11 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_wait_ld();
       float x[32];
       float mc = -INFINITY;
-      const int pos0 = (c_begin + i) * kChunk;
+      const uint32_t vm = misc->vmask[i];  // validity of the chunk's 32 positions
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const int32_t id = pos0 + j < p.k ? __ldg(idx_row + pos0 + j) : -1;
-        x[j] = index_ok(id, E) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+        x[j] = ((vm >> j) & 1u) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
         mc = fmaxf(mc, x[j]);
       }
       float m_new = m_run;
@@ -421,6 +478,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort) report(p.status, DSA_ERR_TIMEOUT);
 }
 
+// Copies the selected latent rows of every query row into a dense buffer,
+// g[(r*k + j), :] = kv[offsets[b] + idx[r][j], :] (zeros where the index is
+// -1 or out of range), using every SM: each warp moves four 1152-byte rows
+// per round with all twelve 16-byte loads of a lane in flight together.  The
+// sparse-MLA kernel then reads whole 32-row chunks with tiled TMA loads.
+__global__ void __launch_bounds__(256)
+    mla_gather_kernel(const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ off,
+                      const int32_t* __restrict__ idx, int T, int k, int64_t total, int64_t kv_rows,
+                      __nv_bfloat16* __restrict__ g) {
+  grid_dependency_wait();  // the indices come from the previous kernel
+  allow_dependents_launch();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_id = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int64_t n_warps = (int64_t)gridDim.x * 8;
+  for (int64_t base = warp_id * 4; base < total; base += n_warps * 4) {
+    uint4 v[4][3];
+    bool ok[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = base + u;
+      ok[u] = false;
+      const uint4* src = nullptr;
+      if (j < total) {
+        const int64_t r = j / k;
+        const int b = (int)(r / T);
+        const int32_t row0 = off[b], E = off[b + 1] - row0;
+        const int32_t id = idx[j];
+        ok[u] = id >= 0 && id < E && row0 >= 0 && (int64_t)row0 + E <= kv_rows;
+        src = reinterpret_cast<const uint4*>(kv + ((int64_t)row0 + (ok[u] ? id : 0)) * kDQK);
+      }
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        const int pc = lane + 32 * c;
+        v[u][c] = (ok[u] && pc < kDQK / 8) ? __ldg(src + pc) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = base + u;
+      if (j >= total) break;
+      uint4* dst = reinterpret_cast<uint4*>(g + j * kDQK);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        const int pc = lane + 32 * c;
+        if (pc < kDQK / 8) dst[pc] = v[u][c];
+      }
+    }
+  }
+}
+
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
 // One CTA of 64 threads per (row, head); thread c owns eight columns and
@@ -537,10 +644,35 @@ int mla_num_splits(int n_rows, int k) {
   return (n_chunks + cps - 1) / cps;
 }
 
-size_t mla_workspace_bytes(int n_rows, int H, int k) {
+// Rows are copied into a dense buffer first when every CTA works through a
+// long list of chunks (its two in-flight gather stages would otherwise keep
+// too few bytes moving per SM) and the buffer stays within L2-sized bounds.
+#ifndef DSA_MLA_PREGATHER_MIN_CHUNKS
+#define DSA_MLA_PREGATHER_MIN_CHUNKS 4
+#endif
+constexpr size_t kPregatherMaxBytes = (size_t)160 << 20;
+
+bool mla_pregather(int n_rows, int k) {
+  const int n_chunks = (k + kChunk - 1) / kChunk;
+  const int ns = mla_num_splits(n_rows, k);
+  const int cps = (n_chunks + ns - 1) / ns;
+  return cps >= DSA_MLA_PREGATHER_MIN_CHUNKS && (size_t)n_rows * k * kDQK * 2 <= kPregatherMaxBytes;
+}
+
+namespace {
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+// Workspace: [split partials bf16][(max, sum) fp32][gathered rows bf16]
+size_t mla_partials_bytes(int n_rows, int H, int k) {
   const int ns = mla_num_splits(n_rows, k);
   if (ns <= 1) return 0;
-  return (size_t)n_rows * ns * H * (kDV * sizeof(__nv_bfloat16) + 2 * sizeof(float));
+  return align256((size_t)n_rows * ns * H * (kDV * sizeof(__nv_bfloat16) + 2 * sizeof(float)));
+}
+}  // namespace
+
+size_t mla_workspace_bytes(int n_rows, int H, int k) {
+  size_t b = mla_partials_bytes(n_rows, H, k);
+  if (mla_pregather(n_rows, k)) b += align256((size_t)n_rows * k * kDQK * sizeof(__nv_bfloat16));
+  return b;
 }
 
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
@@ -565,8 +697,9 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.ws_ml = nullptr;
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
+  p.pregathered = mla_pregather(n_rows, a.k) ? 1 : 0;
   if (ns > 1) {
-    p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);
+    p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);  // partials first
     p.ws_ml = reinterpret_cast<float*>(p.ws_o + (size_t)n_rows * ns * a.H * kDV);
   }
   CUtensorMap tq, tout;
@@ -585,6 +718,17 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     tm_ok = make_tmap_2d(&tout, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDV, (uint64_t)n_rows * a.H, kDV * 4, 32,
                          (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!tm_ok) return DSA_ERR_CUDA;
+  // the dense copy of the selected rows (pre-gathered path only)
+  __nv_bfloat16* gath = nullptr;
+  CUtensorMap tkv = tq;  // unused unless pre-gathered
+  const int64_t g_rows = (int64_t)n_rows * a.k;
+  if (p.pregathered) {
+    gath = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(a.workspace) +
+                                            mla_partials_bytes(n_rows, a.H, a.k));
+    if (!make_tmap_2d(&tkv, gath, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)g_rows, kDQK * 2, 64, kChunk,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+  }
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -592,8 +736,15 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
+  if (p.pregathered) {
+    const int64_t want = (g_rows + 31) / 32;  // CTAs of 8 warps x 4 rows
+    const int gg = (int)std::min<int64_t>(want, (int64_t)device_info().sm_count * 4);
+    if (launch_pdl(mla_gather_kernel, dim3((unsigned)gg), dim3(256), 0, stream, p.kv, p.off, p.idx, p.T, p.k, g_rows,
+                   p.kv_rows, gath) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
   const int64_t grid = (int64_t)n_rows * ns * 2;
-  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p) !=
+  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, tkv, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   if (ns > 1) {

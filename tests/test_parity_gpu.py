@@ -138,6 +138,24 @@ def test_prefill_causal(cuda_device, T, eps, k):
     run_and_check(wl, cuda_device, end_pos=eps)
 
 
+def test_decode_pregathered_rows(cuda_device):
+    """40 sequences, k=512: four chunks per attention CTA, so the selected rows
+    are first copied into a dense buffer and fetched by tiled TMA loads."""
+    from sparse_attention_04_b200 import _lib
+    wl = dsa_inputs.custom("pregather", B=40, end_pos=None, end_pos_range=(600, 3000), topk=512, H=128,
+                           out_dtype="bf16", scale=192 ** -0.5, seed=21)
+    assert _lib.sparse_mla_workspace_size(40, 1, 128, 512) > 40 * 512 * 1152  # holds the dense copy
+    run_and_check(wl, cuda_device, seqs=[0, 7, 23, 39])
+
+
+def test_prefill_pregathered_rows(cuda_device):
+    """Causal prefill of 100 rows with k=512 (the pre-gathered path), with
+    rows before, at and after the point where the causal prefix reaches k."""
+    wl = dsa_inputs.custom("prefill_pg", B=1, T=100, end_pos=None, topk=512, H=128, out_dtype="bf16",
+                           scale=192 ** -0.5, seed=22)
+    run_and_check(wl, cuda_device, end_pos=[560], rows=[0, 1, 49, 50, 51, 52, 98, 99])
+
+
 def test_fp8_small(cuda_device):
     wl = dsa_inputs.custom("fp8s", B=2, end_pos=None, topk=128, H=128, idx_dtype="e4m3", out_dtype="bf16",
                            scale=192 ** -0.5, seed=9, end_pos_range=(1, 1))
