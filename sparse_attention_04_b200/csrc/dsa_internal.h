@@ -76,9 +76,9 @@ struct MlaArgs {
   // wait.  Standalone calls wait first.
   bool early_inputs;
 };
-int mla_num_splits(int n_rows, int k);
+int mla_num_splits(int n_rows, int k, int H);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
-bool mla_pregather(int n_rows, int k);
+bool mla_pregather(int n_rows, int k, int H);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
 
 // Launches `kernel` on `stream` with programmatic stream serialisation, so

@@ -625,23 +625,35 @@ __global__ void __launch_bounds__(64)
 #define DSA_MLA_MIN_CHUNKS_PER_SPLIT 2
 #endif
 
-// Splits of a row's index list: enough CTAs (two per split, one per value
-// half) to cover the SMs when there are few rows, but at least
-// DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split, since every split costs one
-// query-tile load and one 128 x 512 partial (one chunk per split doubles the
-// partials' traffic for a 10% faster gather: a net loss).
+// Splits of a row's index list.  Every split is a pair of CTAs (one per value
+// half, one CTA per SM for shared memory), so n_rows x splits x 2 CTAs run in
+// ceil(that / SMs) waves, each costing its chunks plus about 1.5 chunks of
+// fixed work (query tile, epilogue); every (row, split) partial costs the
+// combine about 0.017 chunk-times at H = 128 (measured on B200).  The split
+// count minimises that estimate, ties going to fewer splits.  At least
+// DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split (one chunk per split doubles
+// the partials' traffic for a 10% faster gather: a net loss).
 static_assert((DSA_MAX_TOPK + kChunk - 1) / kChunk / DSA_MLA_MIN_CHUNKS_PER_SPLIT <= kMaxSplits,
               "the combine holds every split of a row in registers");
 
-int mla_num_splits(int n_rows, int k) {
+int mla_num_splits(int n_rows, int k, int H) {
   const int n_chunks = (k + kChunk - 1) / kChunk;
-  const int sms = device_info().sm_count;
+  const int64_t sms = device_info().sm_count;
   int max_splits = n_chunks / DSA_MLA_MIN_CHUNKS_PER_SPLIT;
   if (max_splits < 1) max_splits = 1;
-  int ns = (sms + n_rows - 1) / n_rows;
-  ns = ns < 1 ? 1 : (ns > max_splits ? max_splits : ns);
-  const int cps = (n_chunks + ns - 1) / ns;
-  return (n_chunks + cps - 1) / cps;
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int ns = 1; ns <= max_splits; ++ns) {
+    const int cps = (n_chunks + ns - 1) / ns;
+    if ((n_chunks + cps - 1) / cps != ns) continue;  // same chunks per split as a smaller count
+    const int64_t waves = ((int64_t)n_rows * ns * 2 + sms - 1) / sms;
+    const int64_t cost = waves * (1000 * (int64_t)cps + 1500) + (ns > 1 ? (int64_t)n_rows * ns * 17 * H / 128 : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  return best;
 }
 
 // Rows are copied into a dense buffer first when every CTA works through a
@@ -652,9 +664,9 @@ int mla_num_splits(int n_rows, int k) {
 #endif
 constexpr size_t kPregatherMaxBytes = (size_t)160 << 20;
 
-bool mla_pregather(int n_rows, int k) {
+bool mla_pregather(int n_rows, int k, int H) {
   const int n_chunks = (k + kChunk - 1) / kChunk;
-  const int ns = mla_num_splits(n_rows, k);
+  const int ns = mla_num_splits(n_rows, k, H);
   const int cps = (n_chunks + ns - 1) / ns;
   return cps >= DSA_MLA_PREGATHER_MIN_CHUNKS && (size_t)n_rows * k * kDQK * 2 <= kPregatherMaxBytes;
 }
@@ -663,7 +675,7 @@ namespace {
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // Workspace: [split partials bf16][(max, sum) fp32][gathered rows bf16]
 size_t mla_partials_bytes(int n_rows, int H, int k) {
-  const int ns = mla_num_splits(n_rows, k);
+  const int ns = mla_num_splits(n_rows, k, H);
   if (ns <= 1) return 0;
   return align256((size_t)n_rows * ns * H * (kDV * sizeof(__nv_bfloat16) + 2 * sizeof(float)));
 }
@@ -671,13 +683,13 @@ size_t mla_partials_bytes(int n_rows, int H, int k) {
 
 size_t mla_workspace_bytes(int n_rows, int H, int k) {
   size_t b = mla_partials_bytes(n_rows, H, k);
-  if (mla_pregather(n_rows, k)) b += align256((size_t)n_rows * k * kDQK * sizeof(__nv_bfloat16));
+  if (mla_pregather(n_rows, k, H)) b += align256((size_t)n_rows * k * kDQK * sizeof(__nv_bfloat16));
   return b;
 }
 
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   const int n_rows = a.B * a.T;
-  const int ns = mla_num_splits(n_rows, a.k);
+  const int ns = mla_num_splits(n_rows, a.k, a.H);
   const int n_chunks = (a.k + kChunk - 1) / kChunk;
   MlaParams p;
   p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
@@ -697,7 +709,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.ws_ml = nullptr;
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
-  p.pregathered = mla_pregather(n_rows, a.k) ? 1 : 0;
+  p.pregathered = mla_pregather(n_rows, a.k, a.H) ? 1 : 0;
   if (ns > 1) {
     p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);  // partials first
     p.ws_ml = reinterpret_cast<float*>(p.ws_o + (size_t)n_rows * ns * a.H * kDV);
