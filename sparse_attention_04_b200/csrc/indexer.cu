@@ -133,6 +133,17 @@ __device__ Split find_split(const int32_t* __restrict__ off, int B, int T, int64
   bad = __any_sync(0xffffffffu, bad);
   Split r{0, 0, 0, bad};
   if (bad) return r;
+  if (nseg == 1) {  // one sequence, one query block: the range in closed form
+    const int len = seg_len<NQ>(off, T, QB, 0);
+    const int64_t total = len + SEG_COST;
+    const int64_t lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+    const int64_t t_lo = max(lo, (int64_t)SEG_COST), t_hi = hi;
+    if (t_hi > t_lo) {
+      r.kt0 = (int)(t_lo - SEG_COST);
+      r.count = (int)(t_hi - t_lo);
+    }
+    return r;
+  }
   int64_t total = 0;
   for (int base = 0; base < nseg; base += 32) {
     const int seg = base + lane;
