@@ -52,13 +52,14 @@ def stage_bytes(wl, end_pos):
     out_b = 4 if wl.out_dtype == "f32" else 2
     T = wl.T
     idx = topk_b = mla = step = 0
+    short = T == 1 and max(end_pos) <= k  # the decode step skips indexer and selection
     for E in end_pos:
         valid_sum = sum(min(E, E - T + t + 1) for t in range(T))
         keff_sum = sum(min(k, E - T + t + 1) for t in range(T))
         idx += E * key_row + T * (qi + 256) + valid_sum * 4
         topk_b += valid_sum * 4 + T * k * 4
         mla += keff_sum * 1152 + T * H * (576 * 2 + 512 * out_b)
-        step += E * key_row + T * (qi + 256) + keff_sum * 1152 + T * H * (576 * 2 + 512 * out_b)
+        step += (0 if short else E * key_row + T * (qi + 256)) + keff_sum * 1152 + T * H * (576 * 2 + 512 * out_b)
     return {"indexer": idx, "topk": topk_b, "sparse_mla": mla, "step": step}
 
 
@@ -318,7 +319,7 @@ def run_native(args, rank, world, local):
     graph_main = capture(G, 0)
     graph_rem = capture(K % G, 0) if K % G else None
     graph_warm = capture(min(W, G), 0) if W > 0 else None
-    launches_per_step = 3 + (1 if _lib.sparse_mla_workspace_size(wl.B, 1, wl.H, wl.topk) > 0 else 0)
+    launches_per_step = _lib.decode_step_launches(wl.B, max_e, wl.topk, wl.H)
 
     # ---- warm-up (untimed)
     for _ in range(max(1, W // max(1, min(W, G)))):
@@ -373,6 +374,11 @@ def run_native(args, rank, world, local):
     names = ["indexer", "topk", "sparse_mla"]
     stage_s = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_prof)) / n_prof / 1e3
                for j, n in enumerate(names)}
+    if max_e <= wl.topk:
+        # short context: the step runs the attention alone (over every
+        # position), so its whole time is the attention stage
+        names = ["sparse_mla"]
+        stage_s = {"sparse_mla": ms_per_step / 1e3}
     dominant = max(stage_s, key=stage_s.get)
     peaks = {}
     try:
@@ -635,7 +641,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "batched", "fp8", "tiny", "prefill4k"])
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "batched", "fp8", "tiny", "prefill4k", "decode2k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--graph-steps", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -121,10 +121,20 @@ int dsa_sparse_mla(const void* q, const void* kv, const int32_t* offsets, const 
 /*
  * The whole decode step (T = 1): stages 1 -> 2 -> 3 on `stream`, scores and
  * indices kept in the workspace.  max_end_pos bounds every end_pos_b (it sets
- * the workspace's score pitch).  Same layouts as above with T = 1.
+ * the workspace's score pitch).  Same layouts as above with T = 1.  When
+ * max_end_pos <= k every sequence keeps all of its positions, so stages 1 and
+ * 2 are skipped (the workspace's scores and indices are then not written) and
+ * stage 3 attends to each whole cache.
  * workspace: dsa_decode_step_workspace_size(B, max_end_pos, k, H) bytes.
  */
 size_t dsa_decode_step_workspace_size(int B, int max_end_pos, int k, int H);
+/*
+ * Kernels one dsa_decode_step call launches for these sizes (the indexer and
+ * the selection are skipped when max_end_pos <= k: every position is then
+ * kept whatever the scores, as the MLX port does below the top-k size).
+ * -1 for invalid sizes.  Useful to budget CUDA-graph nodes.
+ */
+int dsa_decode_step_launches(int B, int max_end_pos, int k, int H);
 int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
                     int idx_dtype, const void* q, const void* kv, const int32_t* offsets, int B,
                     int max_end_pos, int64_t kv_rows, int k, int H, float scale, void* out,

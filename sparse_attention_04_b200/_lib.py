@@ -22,7 +22,8 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
-           "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc")
+           "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc",
+           "dsa_decode_step_launches")
 
 
 class DSAError(RuntimeError):
@@ -47,6 +48,7 @@ def _load():
         "dsa_decode_step": ([P, P, P, P, I, P, P, P, I, I, I64, I, I, F, P, I, P, P, SZ, P, P], I),
         "dsa_decode_step_workspace_layout": ([I, I, I, I, P, P, P, P], I),
         "dsa_sparse_mla_noalloc": ([P, P, P, P, I, I, I, I, F, I64, P, I, P, P, P], I),
+        "dsa_decode_step_launches": ([I, I, I, I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -125,6 +127,11 @@ def sparse_mla_noalloc(q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out,
     _check(lib.dsa_sparse_mla_noalloc(_p(q), _p(kv), _p(offsets), _p(indices), B, T, H, k, float(scale), kv_rows,
                                       _p(out), out_code, _p(lse), _p(status), _stream(stream)),
            "dsa_sparse_mla_noalloc")
+
+
+def decode_step_launches(B, max_end_pos, k, H) -> int:
+    """Kernels one dsa_decode_step launches for these sizes."""
+    return int(lib.dsa_decode_step_launches(B, max_end_pos, k, H))
 
 
 def decode_step_workspace_size(B, max_end_pos, k, H) -> int:

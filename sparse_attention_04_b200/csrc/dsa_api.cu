@@ -100,12 +100,13 @@ int sparse_mla_call(const void* q, const void* kv, const int32_t* offsets, const
                     int H, int k, float scale, int64_t kv_rows, void* out, int out_dtype, float* lse,
                     void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool early_inputs) {
   if (int rc = check_rows(B, T)) return rc;
-  if (!q || !kv || !offsets || !indices || !out) return DSA_ERR_INVALID_ARG;
+  // a NULL index list is the decode step's dense path (every prefix <= k)
+  if (!q || !kv || !offsets || (!indices && !early_inputs) || !out) return DSA_ERR_INVALID_ARG;
   if (H < 1 || k < 1 || k > DSA_MAX_TOPK) return DSA_ERR_INVALID_ARG;
   if (H > DSA_MAX_HEADS) return DSA_ERR_UNSUPPORTED;
   if (out_dtype != DSA_BF16 && out_dtype != DSA_F32) return DSA_ERR_INVALID_ARG;
   if (!(scale == scale) || kv_rows < 1 || kv_rows > ((int64_t)1 << 31) - 1) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(indices))
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || (indices && !aligned16(indices)))
     return DSA_ERR_INVALID_ARG;
   const size_t need = mla_workspace_bytes(B * T, H, k);
   if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace))) return DSA_ERR_WORKSPACE;
@@ -138,6 +139,15 @@ int dsa_decode_step_workspace_layout(int B, int max_end_pos, int k, int H, size_
   return DSA_OK;
 }
 
+int dsa_decode_step_launches(int B, int max_end_pos, int k, int H) {
+  if (B <= 0 || max_end_pos <= 0 || k < 1 || k > DSA_MAX_TOPK || H < 1 || H > DSA_MAX_HEADS) return -1;
+  int n = max_end_pos <= k ? 0 : 2;           // indexer + selection (skipped for short contexts)
+  n += mla_pregather(B, k, H) ? 1 : 0;         // dense copy of the selected rows
+  n += 1;                                      // attention
+  n += mla_num_splits(B, k, H) > 1 ? 1 : 0;    // combine of the split partials
+  return n;
+}
+
 size_t dsa_decode_step_workspace_size(int B, int max_end_pos, int k, int H) {
   size_t m_off = 0;
   if (dsa_decode_step_workspace_layout(B, max_end_pos, k, H, nullptr, nullptr, nullptr, &m_off))
@@ -162,6 +172,16 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* scores = reinterpret_cast<float*>(ws + s_off);
   int32_t* indices = reinterpret_cast<int32_t*>(ws + i_off);
+  if (max_end_pos <= k) {
+    // Every sequence keeps all of its positions whatever the scores
+    // (k_eff = end_pos): the indexer and the selection are skipped and the
+    // attention runs over each whole prefix.  Scores and indices in the
+    // workspace are left unwritten.
+    if (!q_idx || !w || !k_idx || !offsets) return DSA_ERR_INVALID_ARG;
+    if (idx_dtype != DSA_BF16 && idx_dtype != DSA_E4M3) return DSA_ERR_INVALID_ARG;
+    return sparse_mla_call(q, kv, offsets, nullptr, B, 1, H, k, scale, kv_rows, out, out_dtype, lse, ws + m_off,
+                           ws_bytes - m_off, dev_status, stream, true);
+  }
   int rc = dsa_indexer_scores(q_idx, w, k_idx, k_scale, idx_dtype, offsets, B, 1, kv_rows, scores,
                               ld, dev_status, stream);
   if (rc) return rc;

@@ -84,7 +84,14 @@ struct MlaParams {
   int32_t* status;
   int early_inputs;  // q and offsets may be read before the dependency wait
   int pregathered;   // rows already copied into a dense buffer: TMA tile loads
+  int dense;         // no index list: row r attends to its whole causal prefix
 };
+
+// Position selected at slot j of row r: the index list's entry, or (dense
+// mode, every prefix shorter than k) slot j itself while j < the prefix length.
+__device__ __forceinline__ int32_t selected_pos(const int32_t* __restrict__ idx_row, bool dense, int j, int L) {
+  return dense ? (j < L ? j : -1) : idx_row[j];
+}
 
 __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 && idx < E; }
 
@@ -113,7 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t base_row = p.off[b];
   const int E = p.off[b + 1] - base_row;
   const bool geo_ok = base_row >= 0 && E >= p.T && (int64_t)base_row + E <= p.kv_rows;
-  const int32_t* idx_row = p.idx + (int64_t)r * p.k;
+  const int32_t* idx_row = p.dense ? nullptr : p.idx + (int64_t)r * p.k;
+  const bool dense = p.dense != 0;
+  const int L_row = E - p.T + (r - b * p.T) + 1;  // causal prefix of the row
   const int c_begin = sp * p.cps;
   const int n_chunks_total = (p.k + kChunk - 1) / kChunk;
   const int c_end = min(c_begin + p.cps, n_chunks_total);
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (geo_ok) {
     int lv = -1;
     for (int j = c_begin * kChunk + threadIdx.x; j < min(c_end * kChunk, p.k); j += kThreads) {
-      const int32_t id = idx_row[j];
+      const int32_t id = selected_pos(idx_row, dense, j, L_row);
       if (index_ok(id, E)) {
         lv = j;
         atomicOr(&misc->vmask[j / kChunk - c_begin], 1u << (j % kChunk));
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int32_t my_id = -1;
         if (lane < 16) {
           const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
-          my_id = pos < p.k ? idx_row[pos] : -1;
+          my_id = pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
         }
   #pragma unroll 2
         for (int rr = 0; rr < 16; ++rr) {
@@ -487,6 +496,7 @@ __global__ void __launch_bounds__(256)
     mla_gather_kernel(const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ off,
                       const int32_t* __restrict__ idx, int T, int k, int64_t total, int64_t kv_rows,
                       __nv_bfloat16* __restrict__ g) {
+  // idx == nullptr: dense mode, slot j of row r is position j of its prefix
   grid_dependency_wait();  // the indices come from the previous kernel
   allow_dependents_launch();
   const int lane = threadIdx.x & 31;
@@ -504,7 +514,8 @@ __global__ void __launch_bounds__(256)
         const int64_t r = j / k;
         const int b = (int)(r / T);
         const int32_t row0 = off[b], E = off[b + 1] - row0;
-        const int32_t id = idx[j];
+        const int jj = (int)(j - r * k);
+        const int32_t id = idx ? idx[j] : (jj < E - T + (int)(r - (int64_t)b * T) + 1 ? jj : -1);
         ok[u] = id >= 0 && id < E && row0 >= 0 && (int64_t)row0 + E <= kv_rows;
         src = reinterpret_cast<const uint4*>(kv + ((int64_t)row0 + (ok[u] ? id : 0)) * kDQK);
       }
@@ -710,6 +721,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
   p.pregathered = mla_pregather(n_rows, a.k, a.H) ? 1 : 0;
+  p.dense = a.indices == nullptr ? 1 : 0;
   if (ns > 1) {
     p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);  // partials first
     p.ws_ml = reinterpret_cast<float*>(p.ws_o + (size_t)n_rows * ns * a.H * kDV);

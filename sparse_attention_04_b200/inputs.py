@@ -13,6 +13,8 @@ pages print them: "DeepSeek-V3.2-Exp - Keep top-k positions", Indexer.forward;
   batched    B=32, T=1,    end_pos ~ U[8192,131072], topk=2048, H=128, bf16 indexer
   prefill4k  B=1,  T=4096, end_pos=4096 (causal),    topk=2048, H=128, bf16 indexer
   fp8        B=4,  T=1,    end_pos=131072,          topk=2048, H=128, e4m3 indexer
+  decode2k   B=1,  T=1,    end_pos=2048,            topk=2048, H=128, bf16 indexer
+             (short context: every position kept, indexer and selection skipped)
 
 Draw recipe (one torch.Generator seeded with the workload's seed, on the
 device the tensors are made on, draws taken in this order):
@@ -68,6 +70,9 @@ WORKLOADS = {
     "batched": Workload("batched", 32, 1, None, (8192, 131072), 2048, 128, "bf16", 192 ** -0.5, "bf16", 2),
     "prefill4k": Workload("prefill4k", 1, 4096, 4096, None, 2048, 128, "bf16", 192 ** -0.5, "bf16", 3),
     "fp8": Workload("fp8", 4, 1, 131072, None, 2048, 128, "e4m3", 192 ** -0.5, "bf16", 4),
+    # short context: end_pos <= topk, so every position is kept and the decode
+    # step skips the indexer and the selection
+    "decode2k": Workload("decode2k", 1, 1, 2048, None, 2048, 128, "bf16", 192 ** -0.5, "bf16", 5),
 }
 
 

@@ -88,7 +88,11 @@ def run_and_check(wl, device, rows=None, seqs=None, end_pos=None, staged=False, 
     inp = dsa_inputs.make_inputs(wl, device, end_pos=end_pos)
     if mutate:
         mutate(inp)
-    res = api.staged(inp) if (staged or wl.T > 1) else api.decode_step(inp)
+    # a decode step whose every end_pos <= k skips the indexer and the selection
+    # (nothing to compare there): the stages are then checked one by one and
+    # the fused step's dense output separately below
+    short = wl.T == 1 and max(inp.end_pos) <= wl.topk
+    res = api.staged(inp) if (staged or wl.T > 1 or short) else api.decode_step(inp)
     torch.cuda.synchronize()
     assert int(res.status.item()) == 0, _lib_status(res.status)
     seqs = list(range(wl.B)) if seqs is None else seqs
@@ -109,6 +113,12 @@ def run_and_check(wl, device, rows=None, seqs=None, end_pos=None, staged=False, 
     out = res.out.reshape(wl.B * T, wl.H, -1)[glob_rows]
     lse = res.lse.reshape(wl.B * T, wl.H)[glob_rows]
     check_mla(out, lse, gidx, sub, rows)
+    if short and not staged:
+        fused = api.decode_step(inp)
+        torch.cuda.synchronize()
+        assert int(fused.status.item()) == 0, _lib_status(fused.status)
+        check_mla(fused.out.reshape(wl.B, wl.H, -1)[glob_rows], fused.lse.reshape(wl.B, wl.H)[glob_rows], gidx, sub,
+                  rows)
     return res, inp
 
 
@@ -154,6 +164,24 @@ def test_prefill_pregathered_rows(cuda_device):
     wl = dsa_inputs.custom("prefill_pg", B=1, T=100, end_pos=None, topk=512, H=128, out_dtype="bf16",
                            scale=192 ** -0.5, seed=22)
     run_and_check(wl, cuda_device, end_pos=[560], rows=[0, 1, 49, 50, 51, 52, 98, 99])
+
+
+def test_short_context_skips_selection(cuda_device):
+    """Every end_pos <= k: the decode step skips the indexer and the selection
+    (all positions are kept whatever the scores) and attends to each whole
+    prefix; the result must equal the oracle on the full index list."""
+    api = _api()
+    wl = dsa_inputs.custom("short", B=3, end_pos=None, topk=2048, H=128, out_dtype="bf16", scale=192 ** -0.5,
+                           seed=31)
+    inp = dsa_inputs.make_inputs(wl, cuda_device, end_pos=[100, 1500, 2048])
+    res = api.decode_step(inp)
+    torch.cuda.synchronize()
+    assert int(res.status.item()) == 0, _lib_status(res.status)
+    sub = subset(inp, [0, 1, 2])
+    full = torch.full((3, 2048), -1, dtype=torch.int32)
+    for b, E in enumerate(sub.end_pos):
+        full[b, :E] = torch.arange(E, dtype=torch.int32)
+    check_mla(res.out.reshape(3, wl.H, -1), res.lse.reshape(3, wl.H), full, sub, [0, 1, 2])
 
 
 def test_fp8_small(cuda_device):
