@@ -47,8 +47,11 @@ def lib():
         _lib.oracle_bf16_to_f64.restype = D
         _lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         _lib.oracle_e4m3_to_f64.restype = D
+        _lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        _lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        _lib.oracle_quantize_blocks.argtypes = [P, I64, P, P]
         for f in ("oracle_indexer_scores", "oracle_topk", "oracle_sparse_mla", "oracle_dense_mla",
-                  "oracle_num_threads"):
+                  "oracle_num_threads", "oracle_quantize_blocks"):
             getattr(_lib, f).restype = I
     return _lib
 
@@ -156,6 +159,22 @@ def bf16_to_f64(bits: int) -> float:
 
 def e4m3_to_f64(code: int) -> float:
     return lib().oracle_e4m3_to_f64(code)
+
+
+def e4m3_encode(x: float) -> int:
+    """Nearest e4m3 code to the fp32 value x (ties to even, saturating at +-448)."""
+    return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def quantize_blocks(x) -> tuple:
+    """act_quant of [..., 128] bf16 vectors: (uint8 codes [..., 128], fp32 scales [...])."""
+    xb = _bits(x)
+    assert x.shape[-1] == D_I
+    n = xb.numel() // D_I
+    codes = torch.empty(xb.shape, dtype=torch.uint8)
+    scales = torch.empty(xb.shape[:-1], dtype=torch.float32)
+    _check(lib().oracle_quantize_blocks(_ptr(xb), n, _ptr(codes), _ptr(scales)), "quantize_blocks")
+    return codes, scales
 
 
 def num_threads() -> int:

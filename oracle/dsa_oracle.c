@@ -65,6 +65,52 @@ double oracle_e4m3_to_f64(uint8_t v) {
     return s ? -mag : mag;
 }
 
+/* ---- act_quant: block-128 e4m3 quantisation ----------------------------
+ * [Sel] Indexer.forward quantises q and k with act_quant(x, block_size,
+ * scale_fmt) before fp8_index and writes k_cache[start:end] = k_fp8 (its
+ * scale kept beside it).  The pages do not print act_quant.  Reading taken:
+ * one block = one 128-element vector; scale = amax / 448 in fp32 (1 when
+ * amax = 0); each code is the e4m3 value nearest to x / scale (fp32
+ * division), ties to the even code, saturating at +-448.  Codes are found
+ * from the value table the decoder above defines, not from bit tricks. */
+
+static float e4m3_pos_value(int code) { return (float)oracle_e4m3_to_f64((uint8_t)code); }
+
+uint8_t oracle_e4m3_encode(float x) {
+    if (x != x) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const float a = fabsf(x);
+    if (a >= 448.0f) return sign | 0x7E;  /* 0x7E = 448, the largest finite value */
+    int lo = 0;                           /* largest code whose value is <= a     */
+    for (int c = 1; c <= 0x7E; ++c)
+        if (e4m3_pos_value(c) <= a) lo = c;
+    const double vlo = e4m3_pos_value(lo), vhi = e4m3_pos_value(lo + 1);
+    const double dlo = (double)a - vlo, dhi = vhi - (double)a;
+    int c;
+    if (dlo < dhi) c = lo;
+    else if (dhi < dlo) c = lo + 1;
+    else c = (lo & 1) == 0 ? lo : lo + 1; /* tie: the even code */
+    return sign | (uint8_t)c;
+}
+
+/* Quantises n_blocks consecutive 128-element bf16 vectors. */
+int oracle_quantize_blocks(const uint16_t* x, int64_t n_blocks, uint8_t* codes, float* scales) {
+    if (!x || !codes || !scales || n_blocks < 0) return OR_EINVAL;
+    for (int64_t i = 0; i < n_blocks; ++i) {
+        const uint16_t* xb = x + i * OR_DI;
+        float amax = 0.0f;
+        for (int d = 0; d < OR_DI; ++d) {
+            const float v = fabsf((float)oracle_bf16_to_f64(xb[d]));
+            if (v > amax) amax = v;
+        }
+        const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        for (int d = 0; d < OR_DI; ++d)
+            codes[i * OR_DI + d] = oracle_e4m3_encode((float)oracle_bf16_to_f64(xb[d]) / scale);
+        scales[i] = scale;
+    }
+    return OR_OK;
+}
+
 static void row_geometry(const int32_t* off, int T, int64_t r, int* b, int* t,
                          int64_t* E, int64_t* t_abs) {
     *b = (int)(r / T);

@@ -323,3 +323,70 @@ def test_tiny_workload_end_to_end_invariants():
     worst_kept = min(sc[0, s].item() for s in kept)
     assert all(sc[0, s].item() <= worst_kept for s in range(256) if s not in kept)
     assert out.shape == (1, 16, 512) and torch.isfinite(out).all()
+
+
+# ---------------------------------------------------------------- act_quant (e4m3, block 128)
+# The pages call act_quant(x, block_size, scale_fmt) without printing it
+# ("Keep top-k positions", Indexer.forward).  Reading: scale = amax / 448 in
+# fp32, code = nearest e4m3 value of x / scale, ties to the even code,
+# saturating at +-448.  The pins below fix the encoder to the e4m3 value set
+# (through the decoder, itself pinned against torch for every code above) and
+# to hand-worked ties; the block quantiser to its closed forms.
+
+def test_e4m3_encoder_inverts_the_decoder_for_every_finite_code():
+    for code in range(256):
+        if code & 0x7F == 0x7F:
+            continue  # NaN
+        assert oracle.e4m3_encode(oracle.e4m3_to_f64(code)) == code, hex(code)
+
+
+@pytest.mark.parametrize("x,code", [
+    (448.0, 0x7E), (1e6, 0x7E), (-1e6, 0xFE),     # saturation at the largest finite value
+    (1.0625, 0x38),                                # midway 1.0 (0x38) .. 1.125 (0x39): even code
+    (1.1875, 0x3A),                                # midway 1.125 (0x39) .. 1.25 (0x3A): even code
+    (2.0 ** -10, 0x00),                            # midway 0 .. 2^-9 (smallest subnormal): even code
+    (1.5 * 2.0 ** -10, 0x01),                      # nearer 2^-9 than 0
+    (3.0 * 2.0 ** -10, 0x02),                      # midway 2^-9 (0x01) .. 2^-8 (0x02): even code
+    (-0.0, 0x80), (0.0, 0x00), (240.0, 0x77),
+])
+def test_e4m3_encoder_hand_worked_values(x, code):
+    assert oracle.e4m3_encode(x) == code
+
+
+def test_e4m3_encoder_matches_torch_cast_on_random_values():
+    g = torch.Generator().manual_seed(7)
+    x = torch.cat([torch.randn(20000, generator=g) * 30, torch.randn(5000, generator=g) * 1e-3,
+                   (torch.randint(-3000, 3000, (5000,), generator=g).float() + 0.5) / 64])  # many exact ties
+    mine = torch.tensor([oracle.e4m3_encode(float(v)) for v in x], dtype=torch.uint8)
+    ref = x.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(mine, ref)
+
+
+def test_quantize_blocks_closed_forms():
+    g = torch.Generator().manual_seed(8)
+    x = (torch.randn(6, 128, generator=g) * torch.tensor([1e-3, 0.1, 1, 10, 300, 1e4])[:, None]).to(torch.bfloat16)
+    x[2] = 0  # all-zero block
+    codes, scales = oracle.quantize_blocks(x)
+    xf = x.float()
+    amax = xf.abs().amax(dim=1)
+    for i in range(6):
+        if amax[i] == 0:
+            assert scales[i] == 1.0 and torch.all(codes[i] == 0)
+            continue
+        assert scales[i] == (amax[i] / 448.0)  # fp32 division
+        j = int(xf[i].abs().argmax())
+        assert codes[i, j] & 0x7F == 0x7E  # the largest magnitude lands on +-448
+        deq = torch.tensor([oracle.e4m3_to_f64(int(c)) for c in codes[i]], dtype=torch.float64) * float(scales[i])
+        # within half an e4m3 step (relative 2^-4) of the original, or the subnormal spacing
+        err = (deq - xf[i].double()).abs()
+        assert torch.all(err <= torch.maximum(xf[i].double().abs() * 2 ** -4, torch.tensor(2.0 ** -10) * float(scales[i])))
+
+
+def test_quantize_blocks_agrees_with_the_input_generator():
+    """The seeded input module quantises the e4m3 workload with torch ops; the
+    oracle's own quantiser must give the same bytes."""
+    g = torch.Generator().manual_seed(9)
+    x = (torch.randn(64, 128, generator=g) * 2).to(torch.bfloat16)
+    c1, s1 = oracle.quantize_blocks(x)
+    c2, s2 = dsa_inputs.quantize_e4m3_blocks(x)
+    assert torch.equal(c1, c2) and torch.equal(s1, s2)
