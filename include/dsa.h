@@ -142,6 +142,34 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
                     int32_t* dev_status, void* stream);
 
 /*
+ * Cache write of the newest tokens ("Keep top-k positions", Indexer.forward:
+ * k_cache[start:end] = k after act_quant; the latent cache write of the MLA
+ * listing).  For every sequence b and new token t < T, the row
+ * offsets[b+1] - T + t (the sequence's last T rows) of each cache gets:
+ *   kv_cache  <- kv_new[b,t,:576] (bf16 copy)                 if kv_new != NULL
+ *   k_idx_cache <- k_new[b,t,:128]                            if k_new  != NULL
+ *     bf16 (idx_dtype DSA_BF16): copied;
+ *     e4m3 (DSA_E4M3): act_quant of the 128-vector -- scale = amax/448 in fp32
+ *     (1 when amax = 0), codes = nearest e4m3 of x/scale (ties to even,
+ *     saturating), the scale stored in k_scale_cache[row].
+ * k_new [B,T,128] bf16, kv_new [B,T,576] bf16 (device, 16-byte aligned).
+ * Offsets that break the bounds are reported in *dev_status and skipped.
+ */
+int dsa_cache_append(const void* k_new, const void* kv_new, const int32_t* offsets, int B, int T,
+                     int idx_dtype, void* k_idx_cache, float* k_scale_cache, void* kv_cache,
+                     int64_t kv_rows, int32_t* dev_status, void* stream);
+
+/*
+ * act_quant of the indexer queries for the e4m3 path (Indexer.forward:
+ * q_fp8, q_scale = act_quant(q) and weights * q_scale): for every row and
+ * head the 128-vector q_idx[row,h,:] (bf16) becomes e4m3 codes
+ * q_idx_e4m3[row,h,:] with the rule of dsa_cache_append, and
+ * w_out[row,h] = w[row,h] * scale (fp32).  n_rows = B*T.
+ */
+int dsa_quantize_queries(const void* q_idx, const float* w, int n_rows, void* q_idx_e4m3, float* w_out,
+                         void* stream);
+
+/*
  * Stage 3 without a caller workspace.  The paper has no counterpart: this is
  * a convenience of this library, not a step of the method.
  *

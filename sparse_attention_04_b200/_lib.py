@@ -23,7 +23,7 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
            "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc",
-           "dsa_decode_step_launches")
+           "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries")
 
 
 class DSAError(RuntimeError):
@@ -49,6 +49,8 @@ def _load():
         "dsa_decode_step_workspace_layout": ([I, I, I, I, P, P, P, P], I),
         "dsa_sparse_mla_noalloc": ([P, P, P, P, I, I, I, I, F, I64, P, I, P, P, P], I),
         "dsa_decode_step_launches": ([I, I, I, I], I),
+        "dsa_cache_append": ([P, P, P, I, I, I, P, P, P, I64, P, P], I),
+        "dsa_quantize_queries": ([P, P, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -127,6 +129,20 @@ def sparse_mla_noalloc(q, kv, offsets, indices, B, T, H, k, scale, kv_rows, out,
     _check(lib.dsa_sparse_mla_noalloc(_p(q), _p(kv), _p(offsets), _p(indices), B, T, H, k, float(scale), kv_rows,
                                       _p(out), out_code, _p(lse), _p(status), _stream(stream)),
            "dsa_sparse_mla_noalloc")
+
+
+def cache_append(k_new, kv_new, offsets, B, T, k_cache, k_scale, kv_cache, kv_rows, status=None, stream=None):
+    """dsa_cache_append: the newest T tokens' key (e4m3-quantised when the key
+    cache is uint8) and latent rows into each sequence's last T cache rows."""
+    code = DSA_E4M3 if (k_cache is not None and k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)) else DSA_BF16
+    _check(lib.dsa_cache_append(_p(k_new), _p(kv_new), _p(offsets), B, T, code, _p(k_cache), _p(k_scale),
+                                _p(kv_cache), kv_rows, _p(status), _stream(stream)), "dsa_cache_append")
+
+
+def quantize_queries(q_idx, w, n_rows, q_e4m3, w_out, stream=None):
+    """dsa_quantize_queries: e4m3 codes of q_idx and w_out = w * q_scale."""
+    _check(lib.dsa_quantize_queries(_p(q_idx), _p(w), n_rows, _p(q_e4m3), _p(w_out), _stream(stream)),
+           "dsa_quantize_queries")
 
 
 def decode_step_launches(B, max_end_pos, k, H) -> int:
