@@ -427,57 +427,76 @@ def run_native(args, rank, world, local):
 
 
 def run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world):
-    """Per step: host->device copy of the new token's inputs (q_I, w, q and
-    the new key / latent rows, written over the cache's last row), the decode
-    step, device->host copy of the output.  Pinned host buffers, one CUDA graph."""
+    """End to end through the C ABI.  Per step: ONE host->device copy of a
+    pinned staging buffer holding the new token's inputs (q_I in bf16, w, q,
+    the new indexer key and latent row); dsa_cache_append writes the key
+    (e4m3-quantised for the e4m3 cache) and latent row into each sequence's
+    last cache row; for the e4m3 indexer dsa_quantize_queries turns q_I into
+    codes and folds their scales into w; then the decode step; then the
+    device->host copy of the output.  One CUDA graph of steps."""
     import torch
-    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
-    x0 = copies[0]
-    last = x0.offsets[1:].cpu().long() - 1  # last cache row of every sequence
-    h_qi, h_w, h_q = pin(x0.q_idx), pin(x0.w), pin(x0.q)
-    h_k, h_kv = pin(x0.k_idx[last]), pin(x0.kv[last])
-    h_ks = None if x0.k_scale is None else pin(x0.k_scale[last])
+    from sparse_attention_04_b200 import _lib
+    B, H = wl.B, wl.H
+    fp8 = wl.idx_dtype == "e4m3"
+    # staging layout (bytes, 256-aligned sections): q_I bf16 | w | q | k_new | kv_new
+    sizes = [B * 64 * 128 * 2, B * 64 * 4, B * H * 576 * 2, B * 128 * 2, B * 576 * 2]
+    offs, tot = [], 0
+    for sz in sizes:
+        offs.append(tot)
+        tot += (sz + 255) // 256 * 256
+    g = torch.Generator().manual_seed(wl.seed + 100)
+    h_stage = torch.empty(tot, dtype=torch.uint8, pin_memory=True)
+    host_vals = [torch.randn(B, 64, 128, generator=g).to(torch.bfloat16), copies[0].w.cpu().contiguous(),
+                 torch.randn(B, 1, H, 576, generator=g).to(torch.bfloat16),
+                 torch.randn(B, 1, 128, generator=g).to(torch.bfloat16),
+                 torch.randn(B, 1, 576, generator=g).to(torch.bfloat16)]
+    for o, v in zip(offs, host_vals):
+        raw = v.contiguous().view(torch.uint8).reshape(-1)
+        h_stage[o:o + raw.numel()].copy_(raw)
+    d_stage = torch.empty(tot, dtype=torch.uint8, device=dev)
+    view = lambda i, dt, shape: d_stage[offs[i]:offs[i] + sizes[i]].view(dt).view(*shape)
+    d_qi = view(0, torch.bfloat16, (B, 1, 64, 128))
+    d_w = view(1, torch.float32, (B, 1, 64))
+    d_q = view(2, torch.bfloat16, (B, 1, H, 576))
+    d_k = view(3, torch.bfloat16, (B, 1, 128))
+    d_kv = view(4, torch.bfloat16, (B, 1, 576))
+    q8 = torch.empty(B, 1, 64, 128, dtype=torch.uint8, device=dev) if fp8 else None
+    w8 = torch.empty(B, 1, 64, dtype=torch.float32, device=dev) if fp8 else None
     h_out = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
-    last_d = last.to(dev)
-    d_k_row = torch.empty_like(x0.k_idx[last])
-    d_kv_row = torch.empty_like(x0.kv[last])
-    nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
-    h2d = sum(nbytes(t) for t in (h_qi, h_w, h_q, h_k, h_kv, h_ks))
-    d2h = nbytes(h_out)
+    h2d, d2h = tot, h_out.numel() * h_out.element_size()
 
     def e2e_step(i):
         x = copies[i % n_copies]
-        x.q_idx.copy_(h_qi, non_blocking=True)
-        x.w.copy_(h_w, non_blocking=True)
-        x.q.copy_(h_q, non_blocking=True)
-        d_k_row.copy_(h_k, non_blocking=True)
-        d_kv_row.copy_(h_kv, non_blocking=True)
-        x.k_idx.index_copy_(0, last_d, d_k_row)
-        x.kv.index_copy_(0, last_d, d_kv_row)
-        if h_ks is not None:
-            x.k_scale.index_copy_(0, last_d, h_ks.to(dev, non_blocking=True))
-        step(x.q_idx, x.w, x.k_idx, x.k_scale, x.q, x.kv, x.offsets, x.rows, wl.scale)
+        d_stage.copy_(h_stage, non_blocking=True)
+        _lib.cache_append(d_k, d_kv, x.offsets, B, 1, x.k_idx, x.k_scale, x.kv, x.rows, status=step.status)
+        if fp8:
+            _lib.quantize_queries(d_qi, d_w, B, q8, w8)
+            step(q8, w8, x.k_idx, x.k_scale, d_q, x.kv, x.offsets, x.rows, wl.scale)
+        else:
+            step(d_qi, d_w, x.k_idx, x.k_scale, d_q, x.kv, x.offsets, x.rows, wl.scale)
         h_out.copy_(step.out, non_blocking=True)
 
     Ge = min(G, 256)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=stream):
         for i in range(Ge):
             e2e_step(i)
-    g.replay()
+    gr.replay()
     torch.cuda.synchronize()
     reps = max(1, K // Ge)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         ev0.record(stream)
         for _ in range(reps):
-            g.replay()
+            gr.replay()
         ev1.record(stream)
     torch.cuda.synchronize()
     t = reduce_max(ev0.elapsed_time(ev1) / 1e3, world, dev)
     return {"value": round(aggregate_value(reps * Ge, world, t), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "caches stay resident; per step the new token's q_I, w, q, key row and latent row go in, the output comes out"}
+            "note": "caches stay resident; per step one pinned staging buffer (new token's q_I bf16, w, q, key "
+                    "and latent row) goes in, dsa_cache_append writes the new rows (e4m3 keys quantised), the "
+                    "output comes out"}
 
 
 def prefill_indexer_flops(T, E):
