@@ -17,10 +17,11 @@
 //                   (4 warps for decode; 8 for prefill, two per TMEM lane
 //                   quarter, each taking half of the block's queries)
 //   producer warp   TMA: key tiles into a ring of stages, query blocks into
-//                   two slots (reloaded only when the query block changes);
-//                   between loads it writes -inf past each prefill row's
-//                   causal frontier, where no tile is multiplied
+//                   two slots (reloaded only when the query block changes)
 //   MMA warp        TMEM allocator + MMA issuer (one thread)
+//   fill warp       prefill only: -inf past each row's causal frontier, where
+//                   no tile is multiplied (its stores would otherwise delay
+//                   the producer's next load)
 // Key tiles and query blocks land in shared memory in the 128-byte-swizzled
 // K-major layout the MMA descriptors describe; accumulators are double
 // buffered in TMEM so the epilogue of tile i overlaps the MMA of tile i+1.
@@ -51,8 +52,10 @@ struct IdxCfg {
   static constexpr int EPI_WARPS = NQ == 1 ? 4 : 8;
   static constexpr int QPW = NQ * 4 / EPI_WARPS;     // queries per epilogue warp
   static constexpr int SEG_COST = NQ == 1 ? 0 : 1;   // balance units per query block
-  static constexpr int PRODUCER = EPI_WARPS;         // warp indices of the two roles
+  static constexpr int PRODUCER = EPI_WARPS;         // warp indices of the other roles
   static constexpr int MMA_WARP = EPI_WARPS + 1;
+  static constexpr int FILL_WARP = EPI_WARPS + 2;    // prefill only: -inf past the causal frontier
+  static constexpr int ROLE_WARPS = NQ == 1 ? 2 : 3;
   static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
                                    : (2 * N <= 256) ? 256 : 512;
   static constexpr int OFF_K = 0;
@@ -68,7 +71,7 @@ struct IdxCfg {
   static constexpr int USED_BYTES = OFF_MISC + 64;
   static constexpr bool SLACK = USED_BYTES + 1024 <= 232448;
   static constexpr int SMEM_BYTES = USED_BYTES + (SLACK ? 1024 : 0);
-  static constexpr int THREADS = 32 * (EPI_WARPS + 2);
+  static constexpr int THREADS = 32 * (EPI_WARPS + ROLE_WARPS);
   static_assert(NQ % (EPI_WARPS / 4) == 0, "queries split evenly over the warps of a lane quarter");
   static_assert(N <= 256, "MMA N limit");
   static_assert(OFF_Q % 1024 == 0 && OFF_W % 1024 == 0, "swizzle atoms need 1 KiB alignment");
@@ -92,18 +95,23 @@ struct SmemMisc {
 };
 
 // 64-head weighted ReLU sum of one key for one query: sum_h w[h]*max(0, d[h]),
-// d[0..31] in v0 and d[32..63] in v1, on packed two-lane fp32 FMAs.
+// d[0..31] in v0 and d[32..63] in v1, on packed two-lane fp32 arithmetic.
+// The weights are staged halved (exact), and d + |d| is exactly 2*max(0, d)
+// (+0 for d <= 0), so each product (d + |d|) * (w/2) equals max(0, d) * w
+// bit for bit: one packed add and one packed FMA per pair of heads.
 __device__ __forceinline__ float head_sum64(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
-                                            const float* __restrict__ wq) {
+                                            const float* __restrict__ whalf) {
   float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                  make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < 64; c += 4) {
-    const float4 w4 = *reinterpret_cast<const float4*>(wq + c);
+    const float4 w4 = *reinterpret_cast<const float4*>(whalf + c);
     const uint32_t* v = c < 32 ? v0 : v1;
     const int cc = c & 31;
-    const float2 x01 = make_float2(fmaxf(__uint_as_float(v[cc + 0]), 0.f), fmaxf(__uint_as_float(v[cc + 1]), 0.f));
-    const float2 x23 = make_float2(fmaxf(__uint_as_float(v[cc + 2]), 0.f), fmaxf(__uint_as_float(v[cc + 3]), 0.f));
+    const float2 d01 = make_float2(__uint_as_float(v[cc + 0]), __uint_as_float(v[cc + 1]));
+    const float2 d23 = make_float2(__uint_as_float(v[cc + 2]), __uint_as_float(v[cc + 3]));
+    const float2 x01 = __fadd2_rn(d01, make_float2(fabsf(d01.x), fabsf(d01.y)));
+    const float2 x23 = __fadd2_rn(d23, make_float2(fabsf(d23.x), fabsf(d23.y)));
     const int j = (c >> 2) & 1;
     a[2 * j] = __ffma2_rn(x01, make_float2(w4.x, w4.y), a[2 * j]);
     a[2 * j + 1] = __ffma2_rn(x23, make_float2(w4.z, w4.w), a[2 * j + 1]);
@@ -249,38 +257,32 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
   int seg = sp.seg0, kt = sp.kt0;
   int len = count > 0 ? seg_len<NQ>(off, T, QB, seg) : 0;
 
-  if (warp == C::PRODUCER) {
-    // ------------------------------------------------------------ producer (whole warp)
+  if (NQ > 1 && warp == C::FILL_WARP) {
+    // ------------------------------------------------------------ causal fill (whole warp)
     // -inf past the causal frontier of the rows r = blockIdx.x (mod gridDim.x):
     // keys beyond the last tile of a row's query block are never multiplied.
-    // Written 512 bytes per step, a few steps after each load (decode rows
-    // have nothing to fill).
-    const int64_t n_rows = (int64_t)B * T;
-    int64_t f_r = (T > 1 && !sp.bad) ? (int64_t)blockIdx.x : n_rows;
-    int64_t f_pos = 0, f_end = 0;
-    float* f_row = scores;
-    auto fill = [&](int steps) {
-      while (steps > 0) {
-        if (f_pos >= f_end) {
-          if (f_r >= n_rows) return;
-          const int fb = (int)(f_r / T), ft = (int)(f_r - (int64_t)fb * T);
-          f_pos = (int64_t)seg_len<NQ>(off, T, QB, fb * QB + ft / NQ) * 128;
-          f_end = off[fb + 1] - off[fb];
-          f_row = scores + f_r * ld;
-          f_r += gridDim.x;
-          continue;
+    // A warp of its own, 512 bytes per store instruction: kept off the
+    // producer, whose next key-tile load must not wait behind these stores.
+    if (!sp.bad) {
+      const int64_t n_rows = (int64_t)B * T;
+      for (int64_t f_r = blockIdx.x; f_r < n_rows; f_r += gridDim.x) {
+        const int fb = (int)(f_r / T), ft = (int)(f_r - (int64_t)fb * T);
+        const int64_t f_end = off[fb + 1] - off[fb];
+        float* f_row = scores + f_r * ld;
+        // the frontier is a multiple of 128 keys: 16-byte aligned
+        for (int64_t s0 = (int64_t)seg_len<NQ>(off, T, QB, fb * QB + ft / NQ) * 128 + 4 * lane; s0 < f_end;
+             s0 += 128) {
+          if (s0 + 4 <= f_end) {
+            *reinterpret_cast<float4*>(f_row + s0) = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+          } else {
+            for (int j = 0; j < 4; ++j)
+              if (s0 + j < f_end) f_row[s0 + j] = -INFINITY;
+          }
         }
-        const int64_t s0 = f_pos + 4 * lane;  // f_pos is a multiple of 128: 16-byte aligned
-        if (s0 + 4 <= f_end) {
-          *reinterpret_cast<float4*>(f_row + s0) = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        } else {
-          for (int j = 0; j < 4; ++j)
-            if (s0 + j < f_end) f_row[s0 + j] = -INFINITY;
-        }
-        f_pos += 128;
-        --steps;
       }
-    };
+    }
+  } else if (warp == C::PRODUCER) {
+    // ------------------------------------------------------------ producer (whole warp)
     int qord = -1;
     int issued = 0;
     for (int item = 0; item < count; ++item) {
@@ -315,20 +317,19 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
         float* wd = w_s + qs * C::N;
         for (int i = lane; i < C::N; i += 32) {
           const int t = qb * NQ + i / kHI;
-          wd[i] = t < T ? w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
+          // halved (exact for |w| >= 2^-125), see head_sum64
+          wd[i] = t < T ? 0.5f * w[((int64_t)b * T + t) * kHI + (i % kHI)] : 0.f;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(q_full(qs));
       }
       issued = item + 1;
-      fill(4);
       if (++kt == len && item + 1 < count) {
         ++seg;
         kt = 0;
         len = seg_len<NQ>(off, T, QB, seg);
       }
     }
-    if (!*abort) fill(1 << 30);
     if (*abort && lane == 0) {  // let copies already in flight land before the CTA exits
       volatile int never = 0;
       for (int item = max(0, issued - C::KSTAGES); item < issued; ++item)
