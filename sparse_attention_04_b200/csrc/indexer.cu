@@ -56,13 +56,15 @@ struct IdxCfg {
   static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int FILL_WARP = EPI_WARPS + 2;    // prefill only: -inf past the causal frontier
   static constexpr int ROLE_WARPS = NQ == 1 ? 2 : 3;
-  static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
-                                   : (2 * N <= 256) ? 256 : 512;
+  // TMEM accumulators: two for decode (two CTAs share an SM), else as many as
+  // 512 columns hold, so the epilogue's TMEM reads have slack behind the MMA.
+  static constexpr int NACC = NQ == 1 ? 2 : 512 / N;
+  static constexpr int TMEM_COLS = NACC * N;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + KSTAGES * KT_BYTES;
   static constexpr int OFF_W = OFF_Q + QSLOTS * Q_BYTES;
   static constexpr int OFF_BAR = OFF_W + 2 * N * 4;
-  static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 4;
+  static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // The swizzled tiles need 1 KiB alignment.  Where the budget allows, 1 KiB
   // of slack lets the kernel align the base itself; otherwise (the bf16
@@ -117,6 +119,37 @@ __device__ __forceinline__ float head_sum64(const uint32_t (&v0)[32], const uint
     a[2 * j + 1] = __ffma2_rn(x23, make_float2(w4.z, w4.w), a[2 * j + 1]);
   }
   return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+}
+
+// Two queries' head sums of one key at once (the same arithmetic as
+// head_sum64, per query), interleaved so that eight independent packed
+// accumulators keep the FMA pipe busy.
+__device__ __forceinline__ void head_sum64x2(const uint32_t (&va)[2][32], const uint32_t (&vb)[2][32],
+                                             const float* __restrict__ wa, const float* __restrict__ wb,
+                                             float& sa, float& sb) {
+  float2 a[4], c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    a[i] = make_float2(0.f, 0.f);
+    c[i] = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int h = 0; h < 64; h += 4) {
+    const float4 wa4 = *reinterpret_cast<const float4*>(wa + h);
+    const float4 wb4 = *reinterpret_cast<const float4*>(wb + h);
+    const int hi = h >> 5, hh = h & 31;
+    const int j = (h >> 2) & 1;
+    const float2 da01 = make_float2(__uint_as_float(va[hi][hh]), __uint_as_float(va[hi][hh + 1]));
+    const float2 da23 = make_float2(__uint_as_float(va[hi][hh + 2]), __uint_as_float(va[hi][hh + 3]));
+    const float2 db01 = make_float2(__uint_as_float(vb[hi][hh]), __uint_as_float(vb[hi][hh + 1]));
+    const float2 db23 = make_float2(__uint_as_float(vb[hi][hh + 2]), __uint_as_float(vb[hi][hh + 3]));
+    a[2 * j] = __ffma2_rn(__fadd2_rn(da01, make_float2(fabsf(da01.x), fabsf(da01.y))), make_float2(wa4.x, wa4.y), a[2 * j]);
+    a[2 * j + 1] = __ffma2_rn(__fadd2_rn(da23, make_float2(fabsf(da23.x), fabsf(da23.y))), make_float2(wa4.z, wa4.w), a[2 * j + 1]);
+    c[2 * j] = __ffma2_rn(__fadd2_rn(db01, make_float2(fabsf(db01.x), fabsf(db01.y))), make_float2(wb4.x, wb4.y), c[2 * j]);
+    c[2 * j + 1] = __ffma2_rn(__fadd2_rn(db23, make_float2(fabsf(db23.x), fabsf(db23.y))), make_float2(wb4.z, wb4.w), c[2 * j + 1]);
+  }
+  sa = ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+  sb = ((c[0].x + c[0].y) + (c[1].x + c[1].y)) + ((c[2].x + c[2].y) + (c[3].x + c[3].y));
 }
 
 // This CTA's range of work (warp-collective; every lane gets the result).
@@ -211,7 +244,7 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
   auto q_full = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + i); };
   auto q_empty = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 2 + i); };
   auto acc_full = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 4 + i); };
-  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 6 + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * C::KSTAGES + 4 + C::NACC + i); };
   SmemMisc* misc = reinterpret_cast<SmemMisc*>(smem + C::OFF_MISC);
   volatile int* abort = &misc->abort;
 
@@ -229,6 +262,8 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full(i), 2);                  // expect-tx arrival + "weights staged" arrival
       mbar_init(q_empty(i), 1 + C::EPI_WARPS);  // MMA commit + every epilogue warp
+    }
+    for (int i = 0; i < C::NACC; ++i) {
       mbar_init(acc_full(i), 1);
       mbar_init(acc_empty(i), C::EPI_WARPS);
     }
@@ -347,8 +382,8 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
           ++qord;
           if (!mbar_wait(q_full(qord & 1), (qord >> 1) & 1, abort, kWaitLimitNs)) break;
         }
-        const int ab = item & 1;
-        if (!mbar_wait(acc_empty(ab), ((item >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+        const int ab = item % C::NACC;
+        if (!mbar_wait(acc_empty(ab), ((item / C::NACC) & 1) ^ 1, abort, kWaitLimitNs)) break;
         const int st = item % C::KSTAGES;
         if (!mbar_wait(k_full(st), (item / C::KSTAGES) & 1, abort, kWaitLimitNs)) break;
         tc_fence_after();
@@ -378,7 +413,7 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
       if (*abort && issued > 0) {  // MMAs must finish before TMEM is released
         volatile int never = 0;
         const int last = issued - 1;
-        mbar_wait(acc_full(last & 1), (last >> 1) & 1, &never, 10000000ull);
+        mbar_wait(acc_full(last % C::NACC), (last / C::NACC) & 1, &never, 10000000ull);
       }
     }
   } else {
@@ -403,8 +438,8 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
         E = off[b + 1] - base_row;
         start = E - T;
       }
-      const int ab = item & 1;
-      bool ok = mbar_wait(acc_full(ab), (item >> 1) & 1, abort, kWaitLimitNs);
+      const int ab = item % C::NACC;
+      bool ok = mbar_wait(acc_full(ab), (item / C::NACC) & 1, abort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int s = kt * 128 + row;
@@ -422,10 +457,19 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(ab));
+      float sc[C::QPW];
+      if constexpr (C::QPW == 2) {
+        const float* wq = w_s + (qord & 1) * C::N + q_lo * 64;
+        head_sum64x2(v[0], v[1], wq, wq + 64, sc[0], sc[1]);
+      } else {
+#pragma unroll
+        for (int qq = 0; qq < C::QPW; ++qq)
+          sc[qq] = head_sum64(v[qq][0], v[qq][1], w_s + (qord & 1) * C::N + (q_lo + qq) * 64);
+      }
 #pragma unroll
       for (int qq = 0; qq < C::QPW; ++qq) {
         const int q = q_lo + qq;
-        const float score = head_sum64(v[qq][0], v[qq][1], w_s + (qord & 1) * C::N + q * 64) * ksc;
+        const float score = sc[qq] * ksc;
         const int t = qb * NQ + q;
         if (t < T && s < E)
           scores[((int64_t)b * T + t) * ld + s] = (s <= start + t) ? score : -INFINITY;
@@ -476,12 +520,15 @@ int launch_cfg(const IndexerArgs& a, cudaStream_t stream) {
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Queries per prefill block (bf16): N = 64 * kPrefillNQ.
+constexpr int kPrefillNQ = 4;
+
 }  // namespace
 
 int launch_indexer(const IndexerArgs& a, cudaStream_t stream) {
   const bool fp8 = a.idx_dtype == DSA_E4M3;
   if (a.T == 1) return fp8 ? launch_cfg<1, true>(a, stream) : launch_cfg<1, false>(a, stream);
-  return fp8 ? launch_cfg<4, true>(a, stream) : launch_cfg<4, false>(a, stream);
+  return fp8 ? launch_cfg<4, true>(a, stream) : launch_cfg<kPrefillNQ, false>(a, stream);
 }
 
 }  // namespace dsa
