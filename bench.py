@@ -602,7 +602,8 @@ def run_prefill_only(args, rank, world, dev):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded N(0,1) bf16)", "config": {"workload": "prefill4k", "B": 1, "T": 4096,
                                                                      "end_pos": 4096, "heads": 64},
-                "roofline": {k: res[k] for k in ("bound", "achieved", "peak", "unit", "frac", "peak_source")},
+                "roofline": dict({k: res[k] for k in ("bound", "achieved", "peak", "unit", "frac", "peak_source")},
+                                 traffic=load_traffic("prefill4k", "indexer")),
                 "prefill_indexer": res, "clocks": clk}
         print(json.dumps(line), flush=True)
 
