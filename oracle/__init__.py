@@ -50,8 +50,9 @@ def lib():
         _lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         _lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         _lib.oracle_quantize_blocks.argtypes = [P, I64, P, P]
+        _lib.oracle_rope_hadamard.argtypes = [P, I64, I, P, P, P, I64, I, P]
         for f in ("oracle_indexer_scores", "oracle_topk", "oracle_sparse_mla", "oracle_dense_mla",
-                  "oracle_num_threads", "oracle_quantize_blocks"):
+                  "oracle_num_threads", "oracle_quantize_blocks", "oracle_rope_hadamard"):
             getattr(_lib, f).restype = I
     return _lib
 
@@ -175,6 +176,25 @@ def quantize_blocks(x) -> tuple:
     scales = torch.empty(xb.shape[:-1], dtype=torch.float32)
     _check(lib().oracle_quantize_blocks(_ptr(xb), n, _ptr(codes), _ptr(scales)), "quantize_blocks")
     return codes, scales
+
+
+def rope_hadamard(x, pos, rope_cos, rope_sin, round_bf16: bool = True):
+    """Indexer pre-stage of [n_rows, V, 128] bf16 vectors (V vectors share a
+    row's position pos[row]): rotary embedding of the first 64 entries (pairs
+    i, i+32) with the [rope_len, 32] cos/sin tables, then the 128-point
+    Hadamard rotation.  Returns float64 [n_rows, V, 128]; with round_bf16 the
+    two bf16 rounding points of the model are applied (values exactly bf16)."""
+    xb = _bits(x)
+    assert x.dim() == 3 and x.shape[-1] == D_I
+    n_rows, V = x.shape[0], x.shape[1]
+    p = pos.detach().cpu().to(torch.int32).contiguous()
+    c = rope_cos.detach().cpu().float().contiguous()
+    s = rope_sin.detach().cpu().float().contiguous()
+    assert p.numel() == n_rows and c.shape == s.shape and c.shape[1] == 32
+    y = torch.empty((n_rows, V, D_I), dtype=torch.float64)
+    _check(lib().oracle_rope_hadamard(_ptr(xb), n_rows, V, _ptr(p), _ptr(c), _ptr(s), c.shape[0],
+                                      1 if round_bf16 else 0, _ptr(y)), "rope_hadamard")
+    return y
 
 
 def num_threads() -> int:

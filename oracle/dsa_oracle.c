@@ -389,6 +389,75 @@ int oracle_dense_mla(const uint16_t* q, const uint16_t* kv, const int32_t* off, 
     return OR_OK;
 }
 
+/* ---- 5. indexer pre-stage: rotary embedding, then rotate_activation ---- */
+/*
+ * [Sel] Indexer.forward, before act_quant: q (per head) and k are split into
+ * the rope part (the first rope_head_dim = 64 entries) and the rest; the rope
+ * part gets apply_rotary_emb(., freqs_cis, False) -- "rope in indexer is not
+ * interleaved" -- the two parts are joined again, and the 128-vector goes
+ * through rotate_activation.  Neither function is printed on the pages.
+ * Readings taken:
+ *   - not interleaved: rope entry i (i < 32) is paired with entry i + 32,
+ *     and the pair (a, b) becomes (a*cos_i - b*sin_i, a*sin_i + b*cos_i),
+ *     the rotation by the angle whose cos/sin are freqs_cis[pos][i]; the
+ *     table is an input (the pages give no rope base);
+ *   - rotate_activation: the Walsh-Hadamard transform of the 128 entries in
+ *     Sylvester order, H[i][j] = (-1)^popcount(i & j), scaled by 128^-1/2 so
+ *     that it is a rotation (the pages name
+ *     fast_hadamard_transform.hadamard_transform, and a replacement of it by
+ *     a plain linear layer);
+ *   - precision (round_bf16 != 0): q and k are bf16 tensors in the model, so
+ *     the rotated rope part and the transform's output are each rounded to
+ *     the nearest bf16 (ties to even); everything else is exact.  With
+ *     round_bf16 == 0 nothing is rounded.
+ * The transform is the matrix product written out, not a butterfly.
+ * Vector v belongs to row v / vec_per_row, whose position is pos[row].
+ */
+static double round_bf16_f64(double v) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    const double m = frexp(v, &e);             /* v = m * 2^e, 0.5 <= |m| < 1 */
+    return ldexp(nearbyint(ldexp(m, 8)), e - 8); /* 8 significant bits, ties to even */
+}
+
+static int popcount_int(int x) {
+    int c = 0;
+    for (; x; x >>= 1) c += x & 1;
+    return c;
+}
+
+int oracle_rope_hadamard(const uint16_t* x, int64_t n_rows, int vec_per_row, const int32_t* pos,
+                         const float* rope_cos, const float* rope_sin, int64_t rope_len, int round_bf16,
+                         double* y) {
+    if (!x || !pos || !rope_cos || !rope_sin || !y || n_rows < 0 || vec_per_row <= 0 || rope_len <= 0)
+        return OR_EINVAL;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (pos[r] < 0 || pos[r] >= rope_len) return OR_EINVAL;
+    const double scale = 1.0 / sqrt((double)OR_DI);
+#pragma omp parallel for schedule(static)
+    for (int64_t v = 0; v < n_rows * vec_per_row; ++v) {
+        const int64_t p = pos[v / vec_per_row];
+        double a[OR_DI];
+        for (int d = 0; d < OR_DI; ++d) a[d] = oracle_bf16_to_f64(x[v * OR_DI + d]);
+        double u[OR_DI];
+        for (int i = 0; i < 32; ++i) {
+            const double c = rope_cos[p * 32 + i], sn = rope_sin[p * 32 + i];
+            u[i] = a[i] * c - a[i + 32] * sn;
+            u[i + 32] = a[i] * sn + a[i + 32] * c;
+        }
+        for (int d = 64; d < OR_DI; ++d) u[d] = a[d];
+        if (round_bf16)
+            for (int d = 0; d < 64; ++d) u[d] = round_bf16_f64(u[d]);
+        for (int i = 0; i < OR_DI; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < OR_DI; ++j) acc += (popcount_int(i & j) & 1) ? -u[j] : u[j];
+            acc *= scale;
+            y[v * OR_DI + i] = round_bf16 ? round_bf16_f64(acc) : acc;
+        }
+    }
+    return OR_OK;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -390,3 +390,112 @@ def test_quantize_blocks_agrees_with_the_input_generator():
     c1, s1 = oracle.quantize_blocks(x)
     c2, s2 = dsa_inputs.quantize_e4m3_blocks(x)
     assert torch.equal(c1, c2) and torch.equal(s1, s2)
+
+
+# ---------------------------------------------------------------- indexer pre-stage (RoPE + Hadamard)
+
+def _rope_tables(n_pos, base=10000.0):
+    """cos/sin of pos * theta_i, theta_i = base^(-i/32): a freqs_cis table of
+    the usual form (the pages give no base; any table works for the pins)."""
+    theta = base ** (-torch.arange(32, dtype=torch.float64) / 32)
+    ang = torch.arange(n_pos, dtype=torch.float64)[:, None] * theta[None]
+    return torch.cos(ang).float(), torch.sin(ang).float()
+
+
+def _identity_tables(n_pos):
+    return torch.ones(n_pos, 32), torch.zeros(n_pos, 32)
+
+
+def test_rotate_activation_is_the_sylvester_hadamard_matrix():
+    # the transform alone (identity rope) equals scipy's Hadamard matrix / sqrt(128)
+    import scipy.linalg
+    Hm = torch.tensor(scipy.linalg.hadamard(128), dtype=torch.float64) / math.sqrt(128)
+    x = _bf16((5, 3, 128), seed=70)
+    c, s = _identity_tables(4)
+    pos = torch.tensor([0, 1, 2, 3, 0], dtype=torch.int32)
+    y = oracle.rope_hadamard(x, pos, c, s, round_bf16=False)
+    ref = x.double() @ Hm.T
+    assert torch.allclose(y, ref, rtol=0, atol=1e-12)
+
+
+def test_rotate_activation_is_an_involution_and_keeps_the_norm():
+    x = _bf16((4, 2, 128), seed=71, scale=3.0)
+    c, s = _identity_tables(1)
+    pos = torch.zeros(4, dtype=torch.int32)
+    y = oracle.rope_hadamard(x, pos, c, s, round_bf16=False)
+    assert torch.allclose(y.norm(dim=-1), x.double().norm(dim=-1), rtol=1e-13)
+    # H/sqrt(128) is symmetric and orthogonal: applying it twice gives x back
+    import scipy.linalg
+    Hm = torch.tensor(scipy.linalg.hadamard(128), dtype=torch.float64) / math.sqrt(128)
+    assert torch.allclose(y @ Hm, x.double(), atol=1e-12)
+
+
+@pytest.mark.parametrize("i", [0, 5, 31])
+def test_rope_pairs_entry_i_with_entry_i_plus_32(i):
+    # not interleaved: e_i -> cos at i, sin at i+32; e_{i+32} -> -sin at i, cos at i+32
+    import scipy.linalg
+    Hm = torch.tensor(scipy.linalg.hadamard(128), dtype=torch.float64) / math.sqrt(128)
+    c, s = _rope_tables(8)
+    p = 7
+    x = torch.zeros(2, 1, 128)
+    x[0, 0, i] = 1.0
+    x[1, 0, i + 32] = 1.0
+    y = oracle.rope_hadamard(x.to(torch.bfloat16), torch.tensor([p, p], dtype=torch.int32), c, s, round_bf16=False)
+    u = y @ Hm  # undo the (symmetric, orthogonal) transform: the rope output
+    want0 = torch.zeros(128, dtype=torch.float64)
+    want0[i], want0[i + 32] = float(c[p, i]), float(s[p, i])
+    want1 = torch.zeros(128, dtype=torch.float64)
+    want1[i], want1[i + 32] = -float(s[p, i]), float(c[p, i])
+    assert torch.allclose(u[0, 0], want0, atol=1e-12)
+    assert torch.allclose(u[1, 0], want1, atol=1e-12)
+
+
+def test_rope_leaves_the_second_half_alone_and_rotates_by_relative_position():
+    import scipy.linalg
+    Hm = torch.tensor(scipy.linalg.hadamard(128), dtype=torch.float64) / math.sqrt(128)
+    c, s = _rope_tables(64)
+    q = _bf16((1, 1, 128), seed=72)
+    k = _bf16((1, 1, 128), seed=73)
+    uq = oracle.rope_hadamard(q, torch.tensor([10], dtype=torch.int32), c, s, round_bf16=False) @ Hm
+    assert torch.allclose(uq[0, 0, 64:], q[0, 0, 64:].double(), atol=0)  # the non-rope half passes through
+    # <R_p q, R_p' k> depends only on p - p' (the table holds angles pos * theta)
+    dots = []
+    for p, pp in [(10, 3), (20, 13), (40, 33)]:
+        yq = oracle.rope_hadamard(q, torch.tensor([p], dtype=torch.int32), c, s, round_bf16=False)
+        yk = oracle.rope_hadamard(k, torch.tensor([pp], dtype=torch.int32), c, s, round_bf16=False)
+        dots.append(float((yq * yk).sum()))
+    assert max(dots) - min(dots) < 1e-5 * max(1.0, abs(dots[0]))
+
+
+def test_rope_hadamard_bf16_rounding_points():
+    # with rounding: every output is a bf16 value, within the error the two
+    # rounding points allow of the exact result
+    c, s = _rope_tables(32)
+    x = _bf16((6, 4, 128), seed=74)
+    pos = torch.tensor([0, 3, 7, 15, 31, 1], dtype=torch.int32)
+    yr = oracle.rope_hadamard(x, pos, c, s, round_bf16=True)
+    ye = oracle.rope_hadamard(x, pos, c, s, round_bf16=False)
+    assert torch.equal(yr, yr.to(torch.bfloat16).double())
+    rope_l1 = x[..., :64].double().abs().sum(-1, keepdim=True) * 1.42  # |a c - b s| + |a s + b c| <= 1.42 (|a| + |b|)
+    bound = 2.0 ** -8 * ye.abs() + 2.0 ** -9 * rope_l1 / math.sqrt(128) + 1e-12
+    assert bool(((yr - ye).abs() <= bound).all())
+    assert bool(((yr - ye).abs() > 0).any())  # the rounding is really applied
+
+
+def test_rope_hadamard_rejects_positions_outside_the_table():
+    c, s = _rope_tables(4)
+    x = _bf16((2, 1, 128), seed=75)
+    with pytest.raises(ValueError):
+        oracle.rope_hadamard(x, torch.tensor([0, 4], dtype=torch.int32), c, s)
+
+
+def test_rope_hadamard_vectors_of_a_row_share_its_position():
+    # V vectors per row (the 64 heads of a query row) all use pos[row]
+    c, s = _rope_tables(16)
+    x = _bf16((3, 5, 128), seed=76)
+    pos = torch.tensor([2, 9, 15], dtype=torch.int32)
+    y = oracle.rope_hadamard(x, pos, c, s, round_bf16=False)
+    for r in range(3):
+        for v in range(5):
+            one = oracle.rope_hadamard(x[r:r + 1, v:v + 1].contiguous(), pos[r:r + 1], c, s, round_bf16=False)
+            assert torch.equal(y[r, v], one[0, 0])
