@@ -399,6 +399,7 @@ def run_native(args, rank, world, local):
     e2e = run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world)
     del copies
     prefill = None if args.no_prefill else run_prefill(dev, stream, peaks)
+    prestage = None if args.no_prefill else run_prestage(dev, stream, peaks)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
@@ -412,6 +413,8 @@ def run_native(args, rank, world, local):
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * K, "clocks": clk}
     if prefill is not None:
         line["prefill_indexer"] = prefill
+    if prestage is not None:
+        line["indexer_prestage"] = prestage
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = base.to("cpu")
         v, cores, text = time_oracle(wl, cpu, n_steps=3, seconds_per_step_budget=args.cpu_seconds / 3)
@@ -576,6 +579,53 @@ def run_prefill(dev, stream, peaks, reps=20):
             "frac": round(achieved / peak, 4), "peak_source": src,
             "staged_step_us": round(t_all * 1e6, 1),
             "note": "causal lower triangle only; 3 rotating input and score copies"}
+
+
+def run_prestage(dev, stream, peaks, reps=20):
+    """The indexer pre-stage (rotary embedding + Hadamard rotation) over the
+    queries of the causal 4K prefill: 4096 rows x 64 heads of 128 bf16, read
+    and written once (128 MiB per launch), against the HBM copy peak.  Three
+    copies rotate (384 MiB, above 3x L2)."""
+    import torch
+    from sparse_attention_04_b200 import _lib
+    n_rows, V, L, n_copies = 4096, 64, 4096, 3
+    g = torch.Generator(device=dev).manual_seed(3)
+    xs = [torch.randn(n_rows, V, 128, generator=g, device=dev).to(torch.bfloat16) for _ in range(n_copies)]
+    ys = [torch.empty_like(x) for x in xs]
+    pos = torch.arange(n_rows, dtype=torch.int32, device=dev)
+    theta = 10000.0 ** (-torch.arange(32, dtype=torch.float64, device=dev) / 32)
+    ang = torch.arange(L, dtype=torch.float64, device=dev)[:, None] * theta[None]
+    rc, rs = torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            _lib.indexer_prestage(xs[i], pos, rc, rs, y=ys[i], status=status, stream=stream)
+        torch.cuda.synchronize()
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=stream):
+            for i in range(reps):
+                _lib.indexer_prestage(xs[i % n_copies], pos, rc, rs, y=ys[i % n_copies], status=status,
+                                      stream=stream)
+        gph.replay()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        gph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit("prestage: device status " + _lib.status_string(int(status.item())))
+    t = ev0.elapsed_time(ev1) / 1e3 / reps
+    nbytes = 2 * n_rows * V * 128 * 2
+    try:
+        peak, src = float(peaks["hbm_gbs"]), "measured"
+    except Exception:
+        peak, src = 6650.0, "fallback"
+    achieved = nbytes / t / 1e9
+    return {"workload": "prefill4k queries (4096 x 64 x 128 bf16)", "kernel": "rope_hadamard", "bound": "hbm",
+            "us": round(t * 1e6, 2), "bytes": nbytes, "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": src,
+            "vectors_per_s": round(n_rows * V / t, 1)}
 
 
 def run_prefill_only(args, rank, world, dev):

@@ -160,6 +160,24 @@ int dsa_cache_append(const void* k_new, const void* kv_new, const int32_t* offse
                      int64_t kv_rows, int32_t* dev_status, void* stream);
 
 /*
+ * Indexer pre-stage ("Keep top-k positions", Indexer.forward, before
+ * act_quant): for every 128-vector x[r, v, :] (bf16; r < n_rows, v <
+ * vec_per_row -- the 64 heads of a query row, or one key per row)
+ *   1. rotary embedding of the rope part, entries 0..63, not interleaved:
+ *      entry i < 32 pairs with entry i + 32 and (a, b) becomes
+ *      (a*cos - b*sin, a*sin + b*cos), cos/sin = rope_cos/rope_sin[pos[r], i]
+ *      (the freqs_cis table, [rope_len, 32] fp32, row-major); the result is
+ *      rounded to bf16;
+ *   2. rotate_activation: the Walsh-Hadamard transform of the 128 entries in
+ *      Sylvester order, scaled by 128^-1/2, rounded to bf16 into y[r, v, :].
+ * y may equal x.  x, y, rope_cos, rope_sin 16-byte aligned (device).  A
+ * position outside [0, rope_len) leaves that row's vectors untouched and is
+ * reported in *dev_status as DSA_ERR_BAD_INDEX.
+ */
+int dsa_indexer_prestage(const void* x, const int32_t* pos, int n_rows, int vec_per_row, const float* rope_cos,
+                         const float* rope_sin, int rope_len, void* y, int32_t* dev_status, void* stream);
+
+/*
  * act_quant of the indexer queries for the e4m3 path (Indexer.forward:
  * q_fp8, q_scale = act_quant(q) and weights * q_scale): for every row and
  * head the 128-vector q_idx[row,h,:] (bf16) becomes e4m3 codes

@@ -23,7 +23,7 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
            "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc",
-           "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries")
+           "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries", "dsa_indexer_prestage")
 
 
 class DSAError(RuntimeError):
@@ -51,6 +51,7 @@ def _load():
         "dsa_decode_step_launches": ([I, I, I, I], I),
         "dsa_cache_append": ([P, P, P, I, I, I, P, P, P, I64, P, P], I),
         "dsa_quantize_queries": ([P, P, I, P, P, P], I),
+        "dsa_indexer_prestage": ([P, P, I, I, P, P, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -137,6 +138,19 @@ def cache_append(k_new, kv_new, offsets, B, T, k_cache, k_scale, kv_cache, kv_ro
     code = DSA_E4M3 if (k_cache is not None and k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)) else DSA_BF16
     _check(lib.dsa_cache_append(_p(k_new), _p(kv_new), _p(offsets), B, T, code, _p(k_cache), _p(k_scale),
                                 _p(kv_cache), kv_rows, _p(status), _stream(stream)), "dsa_cache_append")
+
+
+def indexer_prestage(x, pos, rope_cos, rope_sin, y=None, status=None, stream=None):
+    """dsa_indexer_prestage on x [n_rows, V, 128] bf16 (V vectors per row share
+    pos[row]): rotary embedding of the rope half, then the Hadamard rotation,
+    into y (a new tensor unless given; y may be x)."""
+    if x.dim() != 3 or x.shape[-1] != 128:
+        raise DSAError(1, "indexer_prestage: x must be [n_rows, V, 128]")
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib.dsa_indexer_prestage(_p(x), _p(pos), x.shape[0], x.shape[1], _p(rope_cos), _p(rope_sin),
+                                    rope_cos.shape[0], _p(y), _p(status), _stream(stream)), "dsa_indexer_prestage")
+    return y
 
 
 def quantize_queries(q_idx, w, n_rows, q_e4m3, w_out, stream=None):
