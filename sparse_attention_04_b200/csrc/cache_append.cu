@@ -131,12 +131,19 @@ __device__ __forceinline__ void rope_hadamard128(float (&e)[64], int32_t p, cons
   // Hadamard butterflies: (u, w) -> (u + w, u - w), u the entry whose bit is clear
 #pragma unroll
   for (int bit = 1; bit < 64; bit <<= 1) {  // local bits 0-5 = entry bits 0-2, 4-6
+    // two butterflies per packed add: j and the next j with the bit clear
+    const int nxt = bit == 1 ? 2 : 1;
 #pragma unroll
     for (int j = 0; j < 64; ++j) {
-      if (j & bit) continue;
-      const float u = e[j], w = e[j | bit];
-      e[j] = u + w;
-      e[j | bit] = u - w;
+      if ((j & bit) || (j & nxt)) continue;
+      const int j2 = j + nxt;
+      const float2 u = make_float2(e[j], e[j2]), w = make_float2(e[j | bit], e[j2 | bit]);
+      const float2 sm = __fadd2_rn(u, w);
+      const float2 df = __ffma2_rn(w, make_float2(-1.f, -1.f), u);
+      e[j] = sm.x;
+      e[j2] = sm.y;
+      e[j | bit] = df.x;
+      e[j2 | bit] = df.y;
     }
   }
   const float sg = hh ? -1.f : 1.f;  // entry bit 3: the pair's upper lane takes u - w
