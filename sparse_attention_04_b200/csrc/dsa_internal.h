@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/dsa.h"
@@ -76,7 +78,35 @@ struct MlaArgs {
   // wait.  Standalone calls wait first.
   bool early_inputs;
 };
+// Kernel parameters of the attention stage (both attention kernels).
+struct MlaParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* kv;
+  const int32_t* off;
+  const int32_t* idx;
+  int T, H, k;
+  int n_splits, cps;  // splits per row, chunks per split
+  float scale_log2;
+  int64_t kv_rows;
+  void* out;
+  int out_bf16;
+  float* lse;
+  __nv_bfloat16* ws_o;  // [rows][splits][H][512] unnormalised partials (n_splits > 1)
+  float* ws_ml;          // [rows][splits][H][2]   their (max, sum)
+  int32_t* status;
+  int early_inputs;  // q and offsets may be read before the dependency wait
+  int pregathered;   // rows already copied into a dense buffer: TMA tile loads
+  int dense;         // no index list: row r attends to its whole causal prefix
+};
+
+// The attention kernel for long index lists (sparse_mla_wide.cu): 64-key
+// chunks, grid of 2 CTAs per (row, split) as the 32-key kernel.
+constexpr int kMlaWideChunk = 64;
+cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout, const CUtensorMap& tkv,
+                                   const MlaParams& p, unsigned grid, cudaStream_t stream);
+
 int mla_num_splits(int n_rows, int k, int H);
+int mla_chunk(int n_rows, int k);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
 bool mla_pregather(int n_rows, int k, int H);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);

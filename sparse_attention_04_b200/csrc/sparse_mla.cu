@@ -68,24 +68,6 @@ struct MlaMisc {
 };
 static_assert(sizeof(MlaMisc) == kMiscBytes, "shared-memory budget of the bookkeeping block");
 
-struct MlaParams {
-  const __nv_bfloat16* kv;
-  const int32_t* off;
-  const int32_t* idx;
-  int T, H, k;
-  int n_splits, cps;  // splits per row, chunks per split
-  float scale_log2;
-  int64_t kv_rows;
-  void* out;
-  int out_bf16;
-  float* lse;
-  __nv_bfloat16* ws_o;  // [rows][splits][H][512] unnormalised partials (n_splits > 1)
-  float* ws_ml;          // [rows][splits][H][2]   their (max, sum)
-  int32_t* status;
-  int early_inputs;  // q and offsets may be read before the dependency wait
-  int pregathered;   // rows already copied into a dense buffer: TMA tile loads
-  int dense;         // no index list: row r attends to its whole causal prefix
-};
 
 // Position selected at slot j of row r: the index list's entry, or (dense
 // mode, every prefix shorter than k) slot j itself while j < the prefix length.
@@ -220,17 +202,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int n_qk = 0, n_pv = 0;
       bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
+      // Descriptors differ only in the start-address field (address >> 4 in
+      // the low 14 bits, no carry below 256 KiB): built once, offset per MMA.
+      const uint64_t qk_a0 = smem_desc(sbase + kOffQ, 16, 1024, kSwizzle128B);
+      const uint64_t qk_b0 = smem_desc(sbase + kOffKv, 16, 1024, kSwizzle128B);
+      const uint64_t pv_a0 = smem_desc(sbase + kOffP, 128, 512, kSwizzleNone);
+      const uint64_t pv_b0 = smem_desc(sbase + kOffKv + (4 * v) * (kChunk * 128), kChunk * 128, 1024, kSwizzle128B);
       // PV of chunk n_pv (its P is in shared memory; p_full has been seen)
       auto issue_pv = [&]() {
         const int j = n_pv;
         tc_fence_after();
-        const uint32_t kvb = sbase + kOffKv + (j & 1) * kKvBytes + (4 * v) * (kChunk * 128);
+        const uint64_t bd0 = pv_b0 + (uint64_t)(((j & 1) * kKvBytes) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < kChunk / 16; ++ks) {
-          const uint64_t ad = smem_desc(sbase + kOffP + ks * 256, 128, 512, kSwizzleNone);
-          const uint64_t bd = smem_desc(kvb + ks * 2048, kChunk * 128, 1024, kSwizzle128B);
-          mma_f16_ss(tmem, ad, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kChunk / 16; ++ks)
+          mma_f16_ss(tmem, pv_a0 + (uint64_t)((ks * 256) >> 4), bd0 + (uint64_t)((ks * 2048) >> 4), kIdescPV,
+                     (j > 0 || ks > 0) ? 1u : 0u);
         tc_commit(pv_done);
         tc_commit(kv_empty(j & 1));
         ++n_pv;
@@ -242,15 +228,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_qk < n_my && n_qk <= n_pv + 1 && mbar_try_wait(kv_full(n_qk & 1), (n_qk >> 1) & 1)) {
           const int st = n_qk & 1;
           tc_fence_after();
-          const uint32_t kvb = sbase + kOffKv + st * kKvBytes;
+          const uint64_t bst = qk_b0 + (uint64_t)((st * kKvBytes) >> 4);
 #pragma unroll 1
           for (int kb = 0; kb < kKB; ++kb) {
+            const uint64_t akb = qk_a0 + (uint64_t)((kb * 16384) >> 4);
+            const uint64_t bkb = bst + (uint64_t)((kb * (kChunk * 128)) >> 4);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc(sbase + kOffQ + kb * 16384 + ks * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(kvb + kb * (kChunk * 128) + ks * 32, 16, 1024, kSwizzle128B);
-              mma_f16_ss(tmem + 256 + 32 * st, ad, bd, kIdescQK, (kb | ks) ? 1u : 0u);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16_ss(tmem + 256 + 32 * st, akb + (uint64_t)ks * 2, bkb + (uint64_t)ks * 2, kIdescQK,
+                         (kb | ks) ? 1u : 0u);
             // a PV whose P is ready is slotted in between the groups of QK
             // MMAs, instead of waiting for the whole (slow, N = 32) QK
             if (n_pv < n_qk && mbar_try_wait(p_full, n_pv & 1)) issue_pv();
@@ -632,25 +618,35 @@ __global__ void __launch_bounds__(64)
 
 }  // namespace
 
-#ifndef DSA_MLA_MIN_CHUNKS_PER_SPLIT
-#define DSA_MLA_MIN_CHUNKS_PER_SPLIT 2
-#endif
+// Which attention kernel a launch uses.  The 64-key kernel halves the QK
+// issue cost per key but starts its first QK only once 64 rows have landed;
+// it wins when the attention CTAs (two per row and split, one per SM) each
+// work through many chunks, i.e. when 2 * rows * 64-key chunks is at least
+// kMlaWideMinChunksPerSm times the SM count (batched decode, prefill).
+constexpr int kMlaWideMinChunksPerSm = 8;
+
+int mla_chunk(int n_rows, int k) {
+  const int64_t n64 = (k + kMlaWideChunk - 1) / kMlaWideChunk;
+  const int64_t sms = device_info().sm_count;
+  return 2 * (int64_t)n_rows * n64 >= kMlaWideMinChunksPerSm * sms ? kMlaWideChunk : kChunk;
+}
 
 // Splits of a row's index list.  Every split is a pair of CTAs (one per value
 // half, one CTA per SM for shared memory), so n_rows x splits x 2 CTAs run in
-// ceil(that / SMs) waves, each costing its chunks plus about 1.5 chunks of
-// fixed work (query tile, epilogue); every (row, split) partial costs the
-// combine about 0.017 chunk-times at H = 128 (measured on B200).  The split
-// count minimises that estimate, ties going to fewer splits.  At least
-// DSA_MLA_MIN_CHUNKS_PER_SPLIT chunks per split (one chunk per split doubles
-// the partials' traffic for a 10% faster gather: a net loss).
-static_assert((DSA_MAX_TOPK + kChunk - 1) / kChunk / DSA_MLA_MIN_CHUNKS_PER_SPLIT <= kMaxSplits,
-              "the combine holds every split of a row in registers");
+// ceil(that / SMs) waves, each costing its chunks (1000 per 32 keys) plus
+// about 1500 of fixed work (query tile, epilogue); every (row, split) partial
+// costs the combine about 17 at H = 128 (measured on B200).  The split count
+// minimises that estimate, ties going to fewer splits, with at least 64 keys
+// per split (fewer keys per split double the partials' traffic for too
+// little gain).
+static_assert(DSA_MAX_TOPK / 64 <= kMaxSplits, "the combine holds every split of a row in registers");
 
 int mla_num_splits(int n_rows, int k, int H) {
-  const int n_chunks = (k + kChunk - 1) / kChunk;
+  const int chunk = mla_chunk(n_rows, k);
+  const int n_chunks = (k + chunk - 1) / chunk;
   const int64_t sms = device_info().sm_count;
-  int max_splits = n_chunks / DSA_MLA_MIN_CHUNKS_PER_SPLIT;
+  int max_splits = n_chunks * chunk / 64;
+  if (max_splits > n_chunks) max_splits = n_chunks;
   if (max_splits < 1) max_splits = 1;
   int best = 1;
   int64_t best_cost = -1;
@@ -658,7 +654,8 @@ int mla_num_splits(int n_rows, int k, int H) {
     const int cps = (n_chunks + ns - 1) / ns;
     if ((n_chunks + cps - 1) / cps != ns) continue;  // same chunks per split as a smaller count
     const int64_t waves = ((int64_t)n_rows * ns * 2 + sms - 1) / sms;
-    const int64_t cost = waves * (1000 * (int64_t)cps + 1500) + (ns > 1 ? (int64_t)n_rows * ns * 17 * H / 128 : 0);
+    const int64_t cost = waves * (1000 * (int64_t)cps * chunk / 32 + 1500) +
+                         (ns > 1 ? (int64_t)n_rows * ns * 17 * H / 128 : 0);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = ns;
@@ -668,18 +665,17 @@ int mla_num_splits(int n_rows, int k, int H) {
 }
 
 // Rows are copied into a dense buffer first when every CTA works through a
-// long list of chunks (its two in-flight gather stages would otherwise keep
+// long list of rows (its two in-flight gather stages would otherwise keep
 // too few bytes moving per SM) and the buffer stays within L2-sized bounds.
-#ifndef DSA_MLA_PREGATHER_MIN_CHUNKS
-#define DSA_MLA_PREGATHER_MIN_CHUNKS 4
-#endif
+constexpr int kPregatherMinKeysPerCta = 128;
 constexpr size_t kPregatherMaxBytes = (size_t)160 << 20;
 
 bool mla_pregather(int n_rows, int k, int H) {
-  const int n_chunks = (k + kChunk - 1) / kChunk;
+  const int chunk = mla_chunk(n_rows, k);
+  const int n_chunks = (k + chunk - 1) / chunk;
   const int ns = mla_num_splits(n_rows, k, H);
   const int cps = (n_chunks + ns - 1) / ns;
-  return cps >= DSA_MLA_PREGATHER_MIN_CHUNKS && (size_t)n_rows * k * kDQK * 2 <= kPregatherMaxBytes;
+  return cps * chunk >= kPregatherMinKeysPerCta && (size_t)n_rows * k * kDQK * 2 <= kPregatherMaxBytes;
 }
 
 namespace {
@@ -701,8 +697,10 @@ size_t mla_workspace_bytes(int n_rows, int H, int k) {
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   const int n_rows = a.B * a.T;
   const int ns = mla_num_splits(n_rows, a.k, a.H);
-  const int n_chunks = (a.k + kChunk - 1) / kChunk;
+  const int chunk = mla_chunk(n_rows, a.k);
+  const int n_chunks = (a.k + chunk - 1) / chunk;
   MlaParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
   p.off = a.offsets;
   p.idx = a.indices;
@@ -749,8 +747,8 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   if (p.pregathered) {
     gath = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(a.workspace) +
                                             mla_partials_bytes(n_rows, a.H, a.k));
-    if (!make_tmap_2d(&tkv, gath, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)g_rows, kDQK * 2, 64, kChunk,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_tmap_2d(&tkv, gath, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)g_rows, kDQK * 2, 64,
+                      (uint32_t)chunk, CU_TENSOR_MAP_SWIZZLE_128B))
       return DSA_ERR_CUDA;
   }
   static bool attr_set = false;
@@ -768,9 +766,11 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
   }
   const int64_t grid = (int64_t)n_rows * ns * 2;
-  if (launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, tkv, p) !=
-      cudaSuccess)
-    return DSA_ERR_CUDA;
+  const cudaError_t e =
+      chunk == kMlaWideChunk
+          ? launch_sparse_mla_wide(tq, tout, tkv, p, (unsigned)grid, stream)
+          : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, tkv, p);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (ns > 1) {
     if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(64), 0, stream,
                    (const __nv_bfloat16*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=

@@ -149,12 +149,12 @@ def test_prefill_causal(cuda_device, T, eps, k):
 
 
 def test_decode_pregathered_rows(cuda_device):
-    """40 sequences, k=512: four chunks per attention CTA, so the selected rows
-    are first copied into a dense buffer and fetched by tiled TMA loads."""
+    """40 sequences, k=512: several chunks per attention CTA, so the selected
+    rows are first copied into a dense buffer and fetched by tiled TMA loads."""
     from sparse_attention_04_b200 import _lib
     wl = dsa_inputs.custom("pregather", B=40, end_pos=None, end_pos_range=(600, 3000), topk=512, H=128,
                            out_dtype="bf16", scale=192 ** -0.5, seed=21)
-    assert _lib.sparse_mla_workspace_size(40, 1, 128, 512) > 40 * 512 * 1152  # holds the dense copy
+    assert _lib.sparse_mla_workspace_size(40, 1, 128, 512) >= 40 * 512 * 1152  # holds the dense copy
     run_and_check(wl, cuda_device, seqs=[0, 7, 23, 39])
 
 
@@ -182,6 +182,29 @@ def test_short_context_skips_selection(cuda_device):
     for b, E in enumerate(sub.end_pos):
         full[b, :E] = torch.arange(E, dtype=torch.int32)
     check_mla(res.out.reshape(3, wl.H, -1), res.lse.reshape(3, wl.H), full, sub, [0, 1, 2])
+
+
+def test_short_context_many_rows(cuda_device):
+    """The short-context path with enough rows that every attention CTA works
+    through many chunks (the 64-key attention kernel), ragged prefixes."""
+    api = _api()
+    wl = dsa_inputs.custom("short_wide", B=24, end_pos=None, topk=2048, H=128, out_dtype="bf16", scale=192 ** -0.5,
+                           seed=32)
+    g = torch.Generator().manual_seed(33)
+    eps = [int(x) for x in torch.randint(64, 2049, (24,), generator=g)]
+    eps[0], eps[1], eps[2] = 1, 2048, 65
+    inp = dsa_inputs.make_inputs(wl, cuda_device, end_pos=eps)
+    res = api.decode_step(inp)
+    torch.cuda.synchronize()
+    assert int(res.status.item()) == 0, _lib_status(res.status)
+    rows = [0, 1, 2, 13, 23]
+    sub = subset(inp, rows)
+    full = torch.full((len(rows), 2048), -1, dtype=torch.int32)
+    for i, E in enumerate(sub.end_pos):
+        full[i, :E] = torch.arange(E, dtype=torch.int32)
+    out = res.out.reshape(24, wl.H, -1)[rows]
+    lse = res.lse.reshape(24, wl.H)[rows]
+    check_mla(out, lse, full, sub, list(range(len(rows))))
 
 
 def test_fp8_small(cuda_device):
