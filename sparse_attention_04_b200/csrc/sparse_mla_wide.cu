@@ -241,6 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // whichever order their inputs arrive: QK(i) once chunk i has landed and
     // softmax(i-1) has read S into registers; PV(j) once softmax(j) has
     // written P(j).  Each PV frees its stage for the load of chunk j + 2.
+    // A QK's 36 MMAs go out back to back (polling for a ready PV between
+    // them measured slower here).
     if (lane == 0) {
       int n_qk = 0, n_pv = 0;
       bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
@@ -285,8 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = 0; ks < 4; ++ks)
               mma_f16_ts(d, tmem + kTmemQ + kb * 32 + ks * 8, bkb + (uint64_t)ks * 2, kIdescQK,
                          (kb | ks) ? 1u : 0u);
-            // a PV whose P is ready is slotted in between the groups of QK MMAs
-            if (n_pv < n_qk && mbar_try_wait(p_full(n_pv & 1), (n_pv >> 1) & 1)) issue_pv();
           }
 #pragma unroll 1
           for (int kb = kQTmemBlocks; kb < kKB; ++kb) {
@@ -295,7 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               mma_f16_ss(d, akb + (uint64_t)ks * 2, bkb + (uint64_t)ks * 2, kIdescQK, 1u);
-            if (n_pv < n_qk && mbar_try_wait(p_full(n_pv & 1), (n_pv >> 1) & 1)) issue_pv();
           }
           tc_commit(s_full);
           ++n_qk;
