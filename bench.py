@@ -430,54 +430,31 @@ def run_native(args, rank, world, local):
 
 
 def run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world):
-    """End to end through the C ABI.  Per step: ONE host->device copy of a
-    pinned staging buffer holding the new token's inputs (q_I in bf16, w, q,
-    the new indexer key and latent row); dsa_cache_append writes the key
-    (e4m3-quantised for the e4m3 cache) and latent row into each sequence's
-    last cache row; for the e4m3 indexer dsa_quantize_queries turns q_I into
-    codes and folds their scales into w; then the decode step; then the
-    device->host copy of the output.  One CUDA graph of steps."""
+    """End to end through the public API (api.HostDecodeStep over the C ABI):
+    per step the new token's inputs go host -> device from pinned memory (q_I
+    in bf16, w, the new indexer key and latent row by a copy kernel, q by the
+    copy engine on a side stream while the indexer and the selection run),
+    dsa_cache_append writes the key (e4m3-quantised for the e4m3 cache) and
+    latent row into each sequence's last cache row, dsa_quantize_queries
+    turns q_I into codes for the e4m3 indexer, the indexer, selection and
+    attention run, and the output comes back device -> host by a copy
+    kernel.  One CUDA graph of steps; each step starts after the previous
+    one has finished."""
     import torch
-    from sparse_attention_04_b200 import _lib
+    from sparse_attention_04_b200 import api
     B, H = wl.B, wl.H
-    fp8 = wl.idx_dtype == "e4m3"
-    # staging layout (bytes, 256-aligned sections): q_I bf16 | w | q | k_new | kv_new
-    sizes = [B * 64 * 128 * 2, B * 64 * 4, B * H * 576 * 2, B * 128 * 2, B * 576 * 2]
-    offs, tot = [], 0
-    for sz in sizes:
-        offs.append(tot)
-        tot += (sz + 255) // 256 * 256
+    hs = api.HostDecodeStep(B, max(copies[0].end_pos), wl.topk, H, wl.idx_dtype, step.out.dtype, dev)
     g = torch.Generator().manual_seed(wl.seed + 100)
-    h_stage = torch.empty(tot, dtype=torch.uint8, pin_memory=True)
-    host_vals = [torch.randn(B, 64, 128, generator=g).to(torch.bfloat16), copies[0].w.cpu().contiguous(),
-                 torch.randn(B, 1, H, 576, generator=g).to(torch.bfloat16),
-                 torch.randn(B, 1, 128, generator=g).to(torch.bfloat16),
-                 torch.randn(B, 1, 576, generator=g).to(torch.bfloat16)]
-    for o, v in zip(offs, host_vals):
-        raw = v.contiguous().view(torch.uint8).reshape(-1)
-        h_stage[o:o + raw.numel()].copy_(raw)
-    d_stage = torch.empty(tot, dtype=torch.uint8, device=dev)
-    view = lambda i, dt, shape: d_stage[offs[i]:offs[i] + sizes[i]].view(dt).view(*shape)
-    d_qi = view(0, torch.bfloat16, (B, 1, 64, 128))
-    d_w = view(1, torch.float32, (B, 1, 64))
-    d_q = view(2, torch.bfloat16, (B, 1, H, 576))
-    d_k = view(3, torch.bfloat16, (B, 1, 128))
-    d_kv = view(4, torch.bfloat16, (B, 1, 576))
-    q8 = torch.empty(B, 1, 64, 128, dtype=torch.uint8, device=dev) if fp8 else None
-    w8 = torch.empty(B, 1, 64, dtype=torch.float32, device=dev) if fp8 else None
-    h_out = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
-    h2d, d2h = tot, h_out.numel() * h_out.element_size()
+    hs.host_q_idx.copy_(torch.randn(B, 1, 64, 128, generator=g).to(torch.bfloat16))
+    hs.host_w.copy_(copies[0].w.cpu().reshape(B, 1, 64))
+    hs.host_q.copy_(torch.randn(B, 1, H, 576, generator=g).to(torch.bfloat16))
+    hs.host_k_new.copy_(torch.randn(B, 1, 128, generator=g).to(torch.bfloat16))
+    hs.host_kv_new.copy_(torch.randn(B, 1, 576, generator=g).to(torch.bfloat16))
+    h2d, d2h = hs.h2d_bytes, hs.d2h_bytes
 
     def e2e_step(i):
         x = copies[i % n_copies]
-        d_stage.copy_(h_stage, non_blocking=True)
-        _lib.cache_append(d_k, d_kv, x.offsets, B, 1, x.k_idx, x.k_scale, x.kv, x.rows, status=step.status)
-        if fp8:
-            _lib.quantize_queries(d_qi, d_w, B, q8, w8)
-            step(q8, w8, x.k_idx, x.k_scale, d_q, x.kv, x.offsets, x.rows, wl.scale)
-        else:
-            step(d_qi, d_w, x.k_idx, x.k_scale, d_q, x.kv, x.offsets, x.rows, wl.scale)
-        h_out.copy_(step.out, non_blocking=True)
+        hs(x.k_idx, x.k_scale, x.kv, x.offsets, x.rows, wl.scale)
 
     Ge = min(G, 256)
     gr = torch.cuda.CUDAGraph()
@@ -497,9 +474,10 @@ def run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world):
     t = reduce_max(ev0.elapsed_time(ev1) / 1e3, world, dev)
     return {"value": round(aggregate_value(reps * Ge, world, t), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "caches stay resident; per step one pinned staging buffer (new token's q_I bf16, w, q, key "
-                    "and latent row) goes in, dsa_cache_append writes the new rows (e4m3 keys quantised), the "
-                    "output comes out"}
+            "note": "caches stay resident; per step the new token's q_I bf16, w, key and latent row go in by a "
+                    "copy kernel over PCIe and q by the copy engine beside the indexer, dsa_cache_append writes "
+                    "the new rows (e4m3 keys quantised), the output comes out by a copy kernel; each step after "
+                    "the previous one"}
 
 
 def prefill_indexer_flops(T, E):

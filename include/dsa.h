@@ -188,6 +188,22 @@ int dsa_quantize_queries(const void* q_idx, const float* w, int n_rows, void* q_
                          void* stream);
 
 /*
+ * Host <-> device copies done by a kernel (not a copy engine), so that a step
+ * fed from host buffers stays one chain of kernel launches on `stream`.
+ * dsa_copy_host_to_device: dst (device) <- src_host; dsa_copy_device_to_host:
+ * dst_host <- src (device).  The host buffer must be page-locked and mapped
+ * into the device's address space as one allocation (cudaHostAlloc, or
+ * torch's pin_memory); this is checked at both ends of the range and anything
+ * else returns DSA_ERR_INVALID_ARG, as do null pointers, pointers not 16-byte
+ * aligned and sizes that are not a multiple of 16.  bytes = 0 does nothing.
+ * The copy waits for the previous kernel in the stream; the host may read
+ * dst_host once the stream has been synchronised.  The caller keeps
+ * ownership of both buffers.
+ */
+int dsa_copy_host_to_device(void* dst, const void* src_host, size_t bytes, void* stream);
+int dsa_copy_device_to_host(void* dst_host, const void* src, size_t bytes, void* stream);
+
+/*
  * Stage 3 without a caller workspace.  The paper has no counterpart: this is
  * a convenience of this library, not a step of the method.
  *

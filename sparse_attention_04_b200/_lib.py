@@ -23,7 +23,8 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
            "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc",
-           "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries", "dsa_indexer_prestage")
+           "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries", "dsa_indexer_prestage",
+           "dsa_copy_host_to_device", "dsa_copy_device_to_host")
 
 
 class DSAError(RuntimeError):
@@ -52,6 +53,8 @@ def _load():
         "dsa_cache_append": ([P, P, P, I, I, I, P, P, P, I64, P, P], I),
         "dsa_quantize_queries": ([P, P, I, P, P, P], I),
         "dsa_indexer_prestage": ([P, P, I, I, P, P, I, P, P, P], I),
+        "dsa_copy_host_to_device": ([P, P, SZ, P], I),
+        "dsa_copy_device_to_host": ([P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -157,6 +160,28 @@ def quantize_queries(q_idx, w, n_rows, q_e4m3, w_out, stream=None):
     """dsa_quantize_queries: e4m3 codes of q_idx and w_out = w * q_scale."""
     _check(lib.dsa_quantize_queries(_p(q_idx), _p(w), n_rows, _p(q_e4m3), _p(w_out), _stream(stream)),
            "dsa_quantize_queries")
+
+
+def _host_p(t: torch.Tensor):
+    if t.is_cuda or not t.is_contiguous():
+        raise DSAError(1, "host buffer must be a contiguous CPU tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def copy_host_to_device(dst, src_host, stream=None):
+    """dsa_copy_host_to_device: dst (CUDA) <- src_host (pinned CPU), by a kernel."""
+    n = src_host.numel() * src_host.element_size()
+    if dst.numel() * dst.element_size() != n:
+        raise DSAError(1, "copy_host_to_device: sizes differ")
+    _check(lib.dsa_copy_host_to_device(_p(dst), _host_p(src_host), n, _stream(stream)), "dsa_copy_host_to_device")
+
+
+def copy_device_to_host(dst_host, src, stream=None):
+    """dsa_copy_device_to_host: dst_host (pinned CPU) <- src (CUDA), by a kernel."""
+    n = src.numel() * src.element_size()
+    if dst_host.numel() * dst_host.element_size() != n:
+        raise DSAError(1, "copy_device_to_host: sizes differ")
+    _check(lib.dsa_copy_device_to_host(_host_p(dst_host), _p(src), n, _stream(stream)), "dsa_copy_device_to_host")
 
 
 def decode_step_launches(B, max_end_pos, k, H) -> int:

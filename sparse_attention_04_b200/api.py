@@ -7,6 +7,7 @@ step of the path runs in the library's kernels.
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Optional
 
 import torch
@@ -49,6 +50,97 @@ class DecodeStep:
                          self.k, self.H, scale, self.out, lse=self.lse, workspace=self.workspace,
                          status=self.status, stream=stream)
         return self.out
+
+
+class HostDecodeStep:
+    """A decode step fed from pinned host memory whose output goes back to
+    pinned host memory: the form a server uses when the new token's
+    projections arrive from the host.
+
+    The caller fills the pinned views host_q_idx [B,1,64,128] bf16, host_w
+    [B,1,64] fp32, host_k_new [B,1,128] bf16, host_kv_new [B,1,576] bf16 and
+    host_q [B,1,H,576] bf16, calls the object with the resident caches, and
+    reads host_out [B,1,H,512] once the stream has been synchronised (and only
+    then refills the inputs).  One call issues on the current stream
+
+        copy kernel (q_I, w, k_new, kv_new) -> dsa_cache_append
+        -> [dsa_quantize_queries for e4m3 keys] -> dsa_indexer_scores
+        -> dsa_topk -> dsa_sparse_mla -> copy kernel (out)
+
+    and on a side stream the transfer of q, the largest input, which only the
+    attention reads: it crosses PCIe while the indexer and the selection run,
+    and the attention waits for it.  Up to Q_KERNEL_COPY_MAX bytes a copy
+    kernel moves q (it finishes within the indexer and leaves the chain free
+    of copy-engine hand-offs, each of which costs several microseconds);
+    above that the copy engine does, so that a long transfer holds no SM
+    while the indexer and the selection want them all.  When every end_pos
+    <= k the attention-only form of dsa_decode_step runs after that wait
+    instead.  Each call starts after everything issued before it on the
+    stream."""
+
+    Q_KERNEL_COPY_MAX = 1 << 20
+
+    def __init__(self, B: int, max_end_pos: int, k: int, H: int, idx_dtype: str = "bf16",
+                 out_dtype=torch.bfloat16, device="cuda"):
+        dev = torch.device(device)
+        self.step = DecodeStep(B, max_end_pos, k, H, out_dtype, dev)
+        self.B, self.max_end_pos, self.k, self.H = B, max_end_pos, k, H
+        self.fp8 = idx_dtype == "e4m3"
+        # one pinned staging buffer for the small inputs, 256-byte aligned sections
+        spec = [(torch.bfloat16, (B, 1, 64, 128)), (torch.float32, (B, 1, 64)),
+                (torch.bfloat16, (B, 1, 128)), (torch.bfloat16, (B, 1, 576))]
+        sizes = [math.prod(shape) * torch.empty((), dtype=dt).element_size() for dt, shape in spec]
+        offs, tot = [], 0
+        for sz in sizes:
+            offs.append(tot)
+            tot += -(-sz // 256) * 256
+        self.host_small = torch.zeros(tot, dtype=torch.uint8, pin_memory=True)
+        self._small = torch.empty(tot, dtype=torch.uint8, device=dev)
+
+        def views(buf):
+            return [buf[o:o + n].view(dt).view(*shape) for o, n, (dt, shape) in zip(offs, sizes, spec)]
+
+        self.host_q_idx, self.host_w, self.host_k_new, self.host_kv_new = views(self.host_small)
+        self._q_idx, self._w, self._k_new, self._kv_new = views(self._small)
+        self.host_q = torch.zeros((B, 1, H, 576), dtype=torch.bfloat16, pin_memory=True)
+        self._q = torch.empty((B, 1, H, 576), dtype=torch.bfloat16, device=dev)
+        self.host_out = torch.zeros(tuple(self.step.out.shape), dtype=out_dtype, pin_memory=True)
+        if self.fp8:
+            self._q8 = torch.empty((B, 1, 64, 128), dtype=torch.uint8, device=dev)
+            self._w8 = torch.empty((B, 1, 64), dtype=torch.float32, device=dev)
+        m_off = _lib.decode_step_workspace_layout(B, max_end_pos, k, H)[3]
+        self._ws_mla = self.step.workspace[m_off:]
+        self._side = torch.cuda.Stream(dev)
+        self.h2d_bytes = tot + self.host_q.numel() * 2
+        self.d2h_bytes = self.host_out.numel() * self.host_out.element_size()
+
+    def __call__(self, k_idx, k_scale, kv, offsets, kv_rows, scale):
+        st, B = self.step, self.B
+        cur = torch.cuda.current_stream()
+        self._side.wait_stream(cur)
+        with torch.cuda.stream(self._side):
+            if self.host_q.numel() * 2 <= self.Q_KERNEL_COPY_MAX:
+                _lib.copy_host_to_device(self._q, self.host_q)
+            else:
+                self._q.copy_(self.host_q, non_blocking=True)
+        _lib.copy_host_to_device(self._small, self.host_small)
+        _lib.cache_append(self._k_new, self._kv_new, offsets, B, 1, k_idx, k_scale, kv, kv_rows, status=st.status)
+        q_idx, w = self._q_idx, self._w
+        if self.fp8:
+            _lib.quantize_queries(q_idx, w, B, self._q8, self._w8)
+            q_idx, w = self._q8, self._w8
+        if self.max_end_pos <= self.k:
+            cur.wait_stream(self._side)
+            st(q_idx, w, k_idx, k_scale, self._q, kv, offsets, kv_rows, scale)
+        else:
+            _lib.indexer_scores(q_idx, w, k_idx, k_scale, offsets, B, 1, kv_rows, st.scores, st.ld,
+                                status=st.status)
+            _lib.topk(st.scores, st.ld, offsets, B, 1, self.k, st.indices, status=st.status)
+            cur.wait_stream(self._side)
+            _lib.sparse_mla(self._q, kv, offsets, st.indices, B, 1, self.H, self.k, scale, kv_rows, st.out,
+                            lse=st.lse, workspace=self._ws_mla, status=st.status)
+        _lib.copy_device_to_host(self.host_out, st.out)
+        return self.host_out
 
 
 def decode_step(inp: Inputs, step: Optional[DecodeStep] = None) -> StepResult:
