@@ -63,7 +63,12 @@ struct IdxCfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + KSTAGES * KT_BYTES;
   static constexpr int OFF_W = OFF_Q + QSLOTS * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_W + 2 * N * 4;
+  // e4m3: a ring of key scales per epilogue thread, fetched KSC_AHEAD tiles
+  // ahead by cp.async
+  static constexpr int KSC_AHEAD = 4;
+  static constexpr int OFF_KSC = OFF_W + 2 * N * 4;
+  static constexpr int KSC_BYTES = FP8 ? KSC_AHEAD * EPI_WARPS * 32 * 4 : 0;
+  static constexpr int OFF_BAR = OFF_KSC + KSC_BYTES;
   static constexpr int NBAR = 2 * KSTAGES + 2 * QSLOTS + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // The swizzled tiles need 1 KiB alignment.  Where the budget allows, 1 KiB
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
     int qord = -1;
     int cur_b = -1, E = 0, start = 0;
     int32_t base_row = 0;
+    float* ksc_ring = reinterpret_cast<float*>(smem + C::OFF_KSC) + threadIdx.x;  // slot i at [i * EPI_WARPS * 32]
     for (int item = 0; item < count; ++item) {
       const int b = seg / QB, qb = seg - b * QB;
       if (item == 0 || kt == 0) {
@@ -438,13 +444,29 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
         E = off[b + 1] - base_row;
         start = E - T;
       }
+      const int s = kt * 128 + row;
+      if constexpr (FP8) {
+        // This thread's key scale for tile item + j goes into ring slot
+        // (item + j) % KSC_AHEAD, one commit group per tile (empty past the
+        // run or the sequence); a run's first tile fetches the slots ahead of
+        // it too.  The HBM latency of the scales then runs behind the tiles
+        // in between instead of after each accumulator.
+        auto fetch = [&](int j) {
+          if (kt + j < len && item + j < count && s + 128 * j < E)
+            cp_async_4(smem_u32(ksc_ring + ((item + j) % C::KSC_AHEAD) * (C::EPI_WARPS * 32)),
+                       k_scale + base_row + s + 128 * j);
+          cp_async_commit();
+        };
+        if (item == 0 || kt == 0) {
+#pragma unroll
+          for (int j = 0; j < C::KSC_AHEAD - 1; ++j) fetch(j);
+        }
+        fetch(C::KSC_AHEAD - 1);
+      }
       const int ab = item % C::NACC;
       bool ok = mbar_wait(acc_full(ab), (item / C::NACC) & 1, abort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int s = kt * 128 + row;
-      float ksc = 1.f;
-      if (FP8 && s < E) ksc = k_scale[base_row + s];
       // every TMEM load of the warp's queries first, then one wait
       uint32_t v[C::QPW][2][32];
 #pragma unroll
@@ -457,6 +479,11 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(ab));
+      float ksc = 1.f;
+      if constexpr (FP8) {
+        cp_async_wait<C::KSC_AHEAD - 1>();  // this tile's group is the oldest still open
+        ksc = ksc_ring[(item % C::KSC_AHEAD) * (C::EPI_WARPS * 32)];
+      }
       float sc[C::QPW];
       if constexpr (C::QPW == 2) {
         const float* wq = w_s + (qord & 1) * C::N + q_lo * 64;
@@ -482,6 +509,7 @@ __global__ void __launch_bounds__(IdxCfg<NQ, FP8>::THREADS, IdxCfg<NQ, FP8>::CTA
         len = seg_len<NQ>(off, T, QB, seg);
       }
     }
+    if constexpr (FP8) cp_async_wait<0>();  // scale fetches past the CTA's last tile
   }
 
   __syncthreads();
