@@ -95,20 +95,18 @@ struct MlaParams {
   float* ws_ml;          // [rows][splits][H][2]   their (max, sum)
   int32_t* status;
   int early_inputs;  // q and offsets may be read before the dependency wait
-  int pregathered;   // rows already copied into a dense buffer: TMA tile loads
   int dense;         // no index list: row r attends to its whole causal prefix
 };
 
 // The attention kernel for long index lists (sparse_mla_wide.cu): 64-key
 // chunks, grid of 2 CTAs per (row, split) as the 32-key kernel.
 constexpr int kMlaWideChunk = 64;
-cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout, const CUtensorMap& tkv,
+cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout,
                                    const MlaParams& p, unsigned grid, cudaStream_t stream);
 
 int mla_num_splits(int n_rows, int k, int H);
 int mla_chunk(int n_rows, int k);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
-bool mla_pregather(int n_rows, int k, int H);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
 
 // Launches `kernel` on `stream` with programmatic stream serialisation, so

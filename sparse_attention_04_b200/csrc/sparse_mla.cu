@@ -79,7 +79,7 @@ __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 &
 
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                      const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
+                      const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mbar_init(q_full, 1);
       for (int i = 0; i < 2; ++i) {
-        mbar_init(kv_full(i), p.pregathered ? 1 : 64);  // TMA expect-tx, or the gather group
+        mbar_init(kv_full(i), 64);  // one arrival per gather thread
         mbar_init(kv_empty(i), 1);
         mbar_init(s_full(i), 1);
       }
@@ -268,66 +268,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- row gather
-    if (p.pregathered) {
-      // The rows were copied into a dense [rows * k, 576] buffer by the gather
-      // kernel: each chunk is 9 tiled TMA loads of 32 rows x 64 columns,
-      // landing in the same swizzled K-major layout.
-      if (threadIdx.x == 128) {
-        int issued = 0;
-        for (int i = 0; i < n_my; ++i) {
-          const int st = i & 1;
-          if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
-          mbar_arrive_expect_tx(kv_full(st), kKvBytes);
-          const int row0 = r * p.k + (c_begin + i) * kChunk;
-          for (int kb = 0; kb < kKB; ++kb)
-            tma_load_2d(sbase + kOffKv + st * kKvBytes + kb * (kChunk * 128), &tm_kv, kb * 64, row0, kv_full(st));
-          issued = i + 1;
-        }
-        if (*abort) {  // let copies in flight land before the CTA exits
-          volatile int never = 0;
-          for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(kv_full(i & 1), (i >> 1) & 1, &never, 10000000ull);
-        }
+    // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
+    // the two groups run independently, so both stages are in flight from
+    // the start and a group waits only for its own copies before it signals.
+    // Each warp copies 16 whole rows, one row at a time, so every copy
+    // instruction reads 512 contiguous bytes of a row.
+    const int pt = threadIdx.x - 128;
+    const int grp = pt >> 6, gw = (pt >> 5) & 1;
+    const __nv_bfloat16* kv = p.kv;
+    for (int i = grp; i < n_my; i += 2) {
+      const int st = i & 1;
+      if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+      int32_t my_id = -1;
+      if (lane < 16) {
+        const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
+        my_id = pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
       }
-    } else {
-      // Warps 4-5 fill stage 0 (even chunks), warps 6-7 stage 1 (odd chunks):
-      // the two groups run independently, so both stages are in flight from
-      // the start and a group waits only for its own copies before it signals.
-      // Each warp copies 16 whole rows, one row at a time, so every copy
-      // instruction reads 512 contiguous bytes of a row.
-      const int pt = threadIdx.x - 128;
-      const int grp = pt >> 6, gw = (pt >> 5) & 1;
-      const __nv_bfloat16* kv = p.kv;
-      for (int i = grp; i < n_my; i += 2) {
-        const int st = i & 1;
-        if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
-        int32_t my_id = -1;
-        if (lane < 16) {
-          const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
-          my_id = pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
-        }
-  #pragma unroll 2
-        for (int rr = 0; rr < 16; ++rr) {
-          const int jr = gw * 16 + rr;
-          const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
-          const bool valid = index_ok(id, E);
-          const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
-          const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
-  #pragma unroll
-          for (int u = 0; u < 3; ++u) {
-            const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
-            if (c < kDQK / 8) {
-              const int kb = c >> 3, cc = c & 7;
-              cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
-            }
+#pragma unroll 2
+      for (int rr = 0; rr < 16; ++rr) {
+        const int jr = gw * 16 + rr;
+        const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
+        const bool valid = index_ok(id, E);
+        const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
+        const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
+          if (c < kDQK / 8) {
+            const int kb = c >> 3, cc = c & 7;
+            cp_async_16(dst_row + kb * (kChunk * 128) + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
           }
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(kv_full(st));
       }
+      cp_async_commit();
       cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(kv_full(st));
     }
+    cp_async_wait<0>();
   } else {
     // -------------------------------------------------------------- softmax + epilogue
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -473,58 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort) report(p.status, DSA_ERR_TIMEOUT);
 }
 
-// Copies the selected latent rows of every query row into a dense buffer,
-// g[(r*k + j), :] = kv[offsets[b] + idx[r][j], :] (zeros where the index is
-// -1 or out of range), using every SM: each warp moves four 1152-byte rows
-// per round with all twelve 16-byte loads of a lane in flight together.  The
-// sparse-MLA kernel then reads whole 32-row chunks with tiled TMA loads.
-__global__ void __launch_bounds__(256)
-    mla_gather_kernel(const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ off,
-                      const int32_t* __restrict__ idx, int T, int k, int64_t total, int64_t kv_rows,
-                      __nv_bfloat16* __restrict__ g) {
-  // idx == nullptr: dense mode, slot j of row r is position j of its prefix
-  grid_dependency_wait();  // the indices come from the previous kernel
-  allow_dependents_launch();
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_id = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int64_t n_warps = (int64_t)gridDim.x * 8;
-  for (int64_t base = warp_id * 4; base < total; base += n_warps * 4) {
-    uint4 v[4][3];
-    bool ok[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t j = base + u;
-      ok[u] = false;
-      const uint4* src = nullptr;
-      if (j < total) {
-        const int64_t r = j / k;
-        const int b = (int)(r / T);
-        const int32_t row0 = off[b], E = off[b + 1] - row0;
-        const int jj = (int)(j - r * k);
-        const int32_t id = idx ? idx[j] : (jj < E - T + (int)(r - (int64_t)b * T) + 1 ? jj : -1);
-        ok[u] = id >= 0 && id < E && row0 >= 0 && (int64_t)row0 + E <= kv_rows;
-        src = reinterpret_cast<const uint4*>(kv + ((int64_t)row0 + (ok[u] ? id : 0)) * kDQK);
-      }
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        const int pc = lane + 32 * c;
-        v[u][c] = (ok[u] && pc < kDQK / 8) ? __ldg(src + pc) : make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t j = base + u;
-      if (j >= total) break;
-      uint4* dst = reinterpret_cast<uint4*>(g + j * kDQK);
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        const int pc = lane + 32 * c;
-        if (pc < kDQK / 8) dst[pc] = v[u][c];
-      }
-    }
-  }
-}
-
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
 // One CTA of 64 threads per (row, head); thread c owns eight columns and
@@ -664,23 +590,9 @@ int mla_num_splits(int n_rows, int k, int H) {
   return best;
 }
 
-// Rows are copied into a dense buffer first when every CTA works through a
-// long list of rows (its two in-flight gather stages would otherwise keep
-// too few bytes moving per SM) and the buffer stays within L2-sized bounds.
-constexpr int kPregatherMinKeysPerCta = 128;
-constexpr size_t kPregatherMaxBytes = (size_t)160 << 20;
-
-bool mla_pregather(int n_rows, int k, int H) {
-  const int chunk = mla_chunk(n_rows, k);
-  const int n_chunks = (k + chunk - 1) / chunk;
-  const int ns = mla_num_splits(n_rows, k, H);
-  const int cps = (n_chunks + ns - 1) / ns;
-  return cps * chunk >= kPregatherMinKeysPerCta && (size_t)n_rows * k * kDQK * 2 <= kPregatherMaxBytes;
-}
-
 namespace {
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-// Workspace: [split partials bf16][(max, sum) fp32][gathered rows bf16]
+// Workspace: [split partials bf16][(max, sum) fp32]
 size_t mla_partials_bytes(int n_rows, int H, int k) {
   const int ns = mla_num_splits(n_rows, k, H);
   if (ns <= 1) return 0;
@@ -689,9 +601,7 @@ size_t mla_partials_bytes(int n_rows, int H, int k) {
 }  // namespace
 
 size_t mla_workspace_bytes(int n_rows, int H, int k) {
-  size_t b = mla_partials_bytes(n_rows, H, k);
-  if (mla_pregather(n_rows, k, H)) b += align256((size_t)n_rows * k * kDQK * sizeof(__nv_bfloat16));
-  return b;
+  return mla_partials_bytes(n_rows, H, k);
 }
 
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
@@ -718,7 +628,6 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.ws_ml = nullptr;
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
-  p.pregathered = mla_pregather(n_rows, a.k, a.H) ? 1 : 0;
   p.dense = a.indices == nullptr ? 1 : 0;
   if (ns > 1) {
     p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);  // partials first
@@ -740,17 +649,6 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     tm_ok = make_tmap_2d(&tout, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDV, (uint64_t)n_rows * a.H, kDV * 4, 32,
                          (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!tm_ok) return DSA_ERR_CUDA;
-  // the dense copy of the selected rows (pre-gathered path only)
-  __nv_bfloat16* gath = nullptr;
-  CUtensorMap tkv = tq;  // unused unless pre-gathered
-  const int64_t g_rows = (int64_t)n_rows * a.k;
-  if (p.pregathered) {
-    gath = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(a.workspace) +
-                                            mla_partials_bytes(n_rows, a.H, a.k));
-    if (!make_tmap_2d(&tkv, gath, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDQK, (uint64_t)g_rows, kDQK * 2, 64,
-                      (uint32_t)chunk, CU_TENSOR_MAP_SWIZZLE_128B))
-      return DSA_ERR_CUDA;
-  }
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -758,18 +656,11 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
       return DSA_ERR_CUDA;
     attr_set = true;
   }
-  if (p.pregathered) {
-    const int64_t want = (g_rows + 31) / 32;  // CTAs of 8 warps x 4 rows
-    const int gg = (int)std::min<int64_t>(want, (int64_t)device_info().sm_count * 4);
-    if (launch_pdl(mla_gather_kernel, dim3((unsigned)gg), dim3(256), 0, stream, p.kv, p.off, p.idx, p.T, p.k, g_rows,
-                   p.kv_rows, gath) != cudaSuccess)
-      return DSA_ERR_CUDA;
-  }
   const int64_t grid = (int64_t)n_rows * ns * 2;
   const cudaError_t e =
       chunk == kMlaWideChunk
-          ? launch_sparse_mla_wide(tq, tout, tkv, p, (unsigned)grid, stream)
-          : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, tkv, p);
+          ? launch_sparse_mla_wide(tq, tout, p, (unsigned)grid, stream)
+          : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (ns > 1) {
     if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(64), 0, stream,

@@ -88,7 +88,7 @@ __device__ __forceinline__ bool index_ok(int32_t idx, int E) { return idx >= 0 &
 
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_mla_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                      const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
+                      const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mbar_init(q_full, 1 + 128);  // TMA bytes of blocks 6-8, and the 128 threads writing blocks 0-5
       for (int s = 0; s < kStages; ++s) {
-        mbar_init(kv_full(s), p.pregathered ? 1 : 128);  // TMA expect-tx, or one cp.async arrival per thread
+        mbar_init(kv_full(s), 128);  // one cp.async arrival per gather thread
         mbar_init(kv_empty(s), 1);
       }
       mbar_init(s_full, 1);
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_qk < n_my && (n_qk == 0 || mbar_try_wait(s_empty, (n_qk - 1) & 1)) &&
             mbar_try_wait(kv_full(n_qk % kStages), (n_qk / kStages) & 1)) {
           const int st = n_qk % kStages;
-          if (!p.pregathered) fence_proxy_async_smem();  // rows written by cp.async, read by the tensor core
+          fence_proxy_async_smem();  // rows written by cp.async, read by the tensor core
           tc_fence_after();
           const uint64_t bst = qk_b0 + (uint64_t)((st * kKvBytes) >> 4);
           const uint32_t d = tmem + kTmemS;
@@ -323,67 +323,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- row gather
-    if (p.pregathered) {
-      // The rows were copied into a dense [rows * k, 576] buffer by the gather
-      // kernel: each chunk is 9 tiled TMA loads of 64 rows x 64 columns,
-      // landing in the same swizzled K-major layout.
-      if (threadIdx.x == 128) {
-        int issued = 0;
-        for (int i = 0; i < n_my; ++i) {
-          const int st = i % kStages;
-          if (!mbar_wait(kv_empty(st), ((i / kStages) & 1) ^ 1, abort, kWaitLimitNs)) break;
-          mbar_arrive_expect_tx(kv_full(st), kKvBytes);
-          const int row0 = r * p.k + (c_begin + i) * kChunk;
-          for (int kb = 0; kb < kKB; ++kb)
-            tma_load_2d(sbase + kOffKv + st * kKvBytes + kb * kBlockBytes, &tm_kv, kb * 64, row0, kv_full(st));
-          issued = i + 1;
-        }
-        if (*abort) {  // let copies in flight land before the CTA exits
-          volatile int never = 0;
-          for (int i = max(0, issued - kStages); i < issued; ++i)
-            mbar_wait(kv_full(i % kStages), (i / kStages) & 1, &never, 10000000ull);
-        }
-      }
-    } else {
-      // Warp 4 + gw copies rows 16gw .. 16gw+15 of every chunk, one row at a
-      // time, so each copy instruction reads 512 contiguous bytes of a row.
-      // Completion is signalled by the copies themselves (cp.async arrival
-      // on the stage's barrier), so both stages are in flight from the start;
-      // the next chunk's indices are read while the current one is issued.
-      const int gw = warp - 4;
-      const __nv_bfloat16* kv = p.kv;
-      auto row_id = [&](int i) -> int32_t {
-        if (lane >= 16) return -1;
-        const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
-        return pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
-      };
-      int32_t next_id = row_id(0);
-      for (int i = 0; i < n_my; ++i) {
-        const int st = i % kStages;
-        const int32_t my_id = next_id;
-        if (i + 1 < n_my) next_id = row_id(i + 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((i / kStages) & 1) ^ 1, abort, kWaitLimitNs)))
-          break;
+    // Warp 4 + gw copies rows 16gw .. 16gw+15 of every chunk, one row at a
+    // time, so each copy instruction reads 512 contiguous bytes of a row.
+    // Completion is signalled by the copies themselves (cp.async arrival
+    // on the stage's barrier), so both stages are in flight from the start;
+    // the next chunk's indices are read while the current one is issued.
+    const int gw = warp - 4;
+    const __nv_bfloat16* kv = p.kv;
+    auto row_id = [&](int i) -> int32_t {
+      if (lane >= 16) return -1;
+      const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
+      return pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
+    };
+    int32_t next_id = row_id(0);
+    for (int i = 0; i < n_my; ++i) {
+      const int st = i % kStages;
+      const int32_t my_id = next_id;
+      if (i + 1 < n_my) next_id = row_id(i + 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((i / kStages) & 1) ^ 1, abort, kWaitLimitNs)))
+        break;
 #pragma unroll 2
-        for (int rr = 0; rr < 16; ++rr) {
-          const int jr = gw * 16 + rr;
-          const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
-          const bool valid = index_ok(id, E);
-          const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
-          const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
+      for (int rr = 0; rr < 16; ++rr) {
+        const int jr = gw * 16 + rr;
+        const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
+        const bool valid = index_ok(id, E);
+        const __nv_bfloat16* src = valid ? kv + ((int64_t)base_row + id) * kDQK : kv;
+        const uint32_t dst_row = sbase + kOffKv + st * kKvBytes + (jr >> 3) * 1024 + (jr & 7) * 128;
 #pragma unroll
-          for (int u = 0; u < 3; ++u) {
-            const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
-            if (c < kDQK / 8) {
-              const int kb = c >> 3, cc = c & 7;
-              cp_async_16(dst_row + kb * kBlockBytes + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
-            }
+        for (int u = 0; u < 3; ++u) {
+          const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
+          if (c < kDQK / 8) {
+            const int kb = c >> 3, cc = c & 7;
+            cp_async_16(dst_row + kb * kBlockBytes + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
           }
         }
-        cp_async_mbar_arrive(kv_full(st));
       }
-      cp_async_wait<0>();
+      cp_async_mbar_arrive(kv_full(st));
     }
+    cp_async_wait<0>();
   } else {
     // -------------------------------------------------------------- softmax + epilogue
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -541,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout, const CUtensorMap& tkv,
+cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout,
                                    const MlaParams& p, unsigned grid, cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
@@ -550,7 +527,7 @@ cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tou
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(sparse_mla_wide_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tout, tkv, p);
+  return launch_pdl(sparse_mla_wide_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p);
 }
 
 }  // namespace dsa

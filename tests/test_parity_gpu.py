@@ -148,18 +148,16 @@ def test_prefill_causal(cuda_device, T, eps, k):
     run_and_check(wl, cuda_device, end_pos=eps)
 
 
-def test_decode_pregathered_rows(cuda_device):
-    """40 sequences, k=512: several chunks per attention CTA, so the selected
-    rows are first copied into a dense buffer and fetched by tiled TMA loads."""
-    from sparse_attention_04_b200 import _lib
-    wl = dsa_inputs.custom("pregather", B=40, end_pos=None, end_pos_range=(600, 3000), topk=512, H=128,
+def test_decode_many_chunks_per_cta(cuda_device):
+    """40 sequences, k=512: several 32-key chunks per attention CTA, each
+    attention CTA's two gather stages cycling through its list."""
+    wl = dsa_inputs.custom("many_chunks", B=40, end_pos=None, end_pos_range=(600, 3000), topk=512, H=128,
                            out_dtype="bf16", scale=192 ** -0.5, seed=21)
-    assert _lib.sparse_mla_workspace_size(40, 1, 128, 512) >= 40 * 512 * 1152  # holds the dense copy
     run_and_check(wl, cuda_device, seqs=[0, 7, 23, 39])
 
 
-def test_prefill_pregathered_rows(cuda_device):
-    """Causal prefill of 100 rows with k=512 (the pre-gathered path), with
+def test_prefill_many_chunks_per_cta(cuda_device):
+    """Causal prefill of 100 rows with k=512 (several chunks per CTA), with
     rows before, at and after the point where the causal prefix reaches k."""
     wl = dsa_inputs.custom("prefill_pg", B=1, T=100, end_pos=None, topk=512, H=128, out_dtype="bf16",
                            scale=192 ** -0.5, seed=22)
