@@ -144,19 +144,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_dependency_wait();  // the indices come from the previous kernel
   allow_dependents_launch();
 
-  // ---- how many chunks of this split hold a selected row
+  // ---- how many chunks of this split hold a selected row.  Each warp owns
+  // whole chunks: it loads all their indices first (one L2 round trip), then
+  // builds each chunk's validity mask with ballots, so no shared-memory
+  // atomics contend on a chunk's mask word.
   if (geo_ok) {
-    int lv = -1;
-    for (int j = c_begin * kChunk + threadIdx.x; j < min(c_end * kChunk, p.k); j += kThreads) {
-      const int32_t id = selected_pos(idx_row, dense, j, L_row);
-      if (index_ok(id, E)) {
-        lv = j;
-        atomicOr(&misc->vmask[j / kChunk - c_begin], 1u << (j % kChunk));
-      } else if (id != -1) {
-        report(p.status, DSA_ERR_BAD_INDEX);
+    constexpr int kWarps = kThreads / 32, kPerWarp = (kMaxChunks + kWarps - 1) / kWarps;
+    const int n_ch = c_end - c_begin;
+    int32_t ids[kPerWarp][kChunk / 32];
+#pragma unroll
+    for (int u = 0; u < kPerWarp; ++u)
+#pragma unroll
+      for (int hh = 0; hh < kChunk / 32; ++hh) {
+        const int c = warp + kWarps * u, j = (c_begin + c) * kChunk + 32 * hh + lane;
+        ids[u][hh] = (c < n_ch && j < p.k) ? selected_pos(idx_row, dense, j, L_row) : -1;
       }
+    int lv = -1;
+#pragma unroll
+    for (int u = 0; u < kPerWarp; ++u) {
+      const int c = warp + kWarps * u;
+      if (c >= n_ch) break;  // uniform over the warp
+      uint32_t m = 0;
+#pragma unroll
+      for (int hh = 0; hh < kChunk / 32; ++hh) {
+        const bool valid = index_ok(ids[u][hh], E);
+        if (!valid && ids[u][hh] != -1) report(p.status, DSA_ERR_BAD_INDEX);
+        m |= static_cast<uint32_t>(__ballot_sync(0xffffffffu, valid)) << (32 * hh);
+      }
+      if (lane == 0) misc->vmask[c] = m;
+      if (m) lv = (c_begin + c) * kChunk + 31 - __clz((int)m);
     }
-    if (lv >= 0) atomicMax(&misc->last_valid, lv);
+    if (lane == 0 && lv >= 0) atomicMax(&misc->last_valid, lv);
   } else if (threadIdx.x == 0) {
     report(p.status, DSA_ERR_BAD_OFFSETS);
   }
