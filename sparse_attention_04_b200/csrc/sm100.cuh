@@ -130,6 +130,15 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int
                : "memory");
 }
 
+// ---------------------------------------------------------------- math
+// 2^x by the ex2.approx.ftz.f32 instruction (relative error about 2^-22,
+// subnormal results flushed to zero; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- cp.async
 
 // 16-byte async copy; src_bytes = 0 writes zeros (nothing is read).

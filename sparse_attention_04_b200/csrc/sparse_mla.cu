@@ -340,10 +340,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       float x[32];
       float mc = -INFINITY;
       const uint32_t vm = misc->vmask[i];  // validity of the chunk's 32 positions
+      if (vm == ~0u) {  // every position valid (the common case): scale in pairs
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x[j] = ((vm >> j) & 1u) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
-        mc = fmaxf(mc, x[j]);
+        for (int j = 0; j < 32; j += 2) {
+          const float2 x2 = __fmul2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
+                                       make_float2(p.scale_log2, p.scale_log2));
+          x[j] = x2.x;
+          x[j + 1] = x2.y;
+          mc = fmaxf(mc, fmaxf(x2.x, x2.y));
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x[j] = ((vm >> j) & 1u) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+          mc = fmaxf(mc, x[j]);
+        }
       }
       float m_new = m_run;
       bool resc = false;
@@ -352,17 +363,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_new = mc;
       }
       const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
+      // p = 2^(x - m) (masked positions carry x = -inf, so p = +0), rounded
+      // to bf16 for P.V; the running sum adds the same rounded values
       uint32_t pk[16];
-      float l_chunk = 0.f;
+      float2 l2 = make_float2(0.f, 0.f);
+      const float m_sub = m_new == -INFINITY ? 0.f : m_new;  // nothing valid yet: every x is -inf
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
-        const float p0 = x[j] == -INFINITY ? 0.f : exp2f(x[j] - m_new);
-        const float p1 = x[j + 1] == -INFINITY ? 0.f : exp2f(x[j + 1] - m_new);
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        const float2 back = __bfloat1622float2(pb);
-        l_chunk += back.x + back.y;
+        const float2 d = __fadd2_rn(make_float2(x[j], x[j + 1]), make_float2(-m_sub, -m_sub));
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(ex2_approx(d.x), ex2_approx(d.y));
+        l2 = __fadd2_rn(l2, __bfloat1622float2(pb));
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&pb);
       }
+      const float l_chunk = l2.x + l2.y;
       if (i > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort, kWaitLimitNs));
         if (!ok) break;

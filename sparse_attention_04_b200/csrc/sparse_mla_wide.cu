@@ -397,11 +397,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(s_empty);  // S is in registers: the next chunk's QK may overwrite it
       const unsigned long long vm = misc->vmask[i];  // validity of the chunk's 64 positions
       float mc = -INFINITY;
+      if (vm == ~0ull) {  // every position valid (the common case): scale in pairs
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float xj = ((vm >> j) & 1ull) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
-        sv[j] = __float_as_uint(xj);
-        mc = fmaxf(mc, xj);
+        for (int j = 0; j < 64; j += 2) {
+          const float2 x2 = __fmul2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
+                                       make_float2(p.scale_log2, p.scale_log2));
+          sv[j] = __float_as_uint(x2.x);
+          sv[j + 1] = __float_as_uint(x2.y);
+          mc = fmaxf(mc, fmaxf(x2.x, x2.y));
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float xj = ((vm >> j) & 1ull) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+          sv[j] = __float_as_uint(xj);
+          mc = fmaxf(mc, xj);
+        }
       }
       float m_new = m_run;
       bool resc = false;
@@ -410,18 +421,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_new = mc;
       }
       const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
+      // p = 2^(x - m) (masked positions carry x = -inf, so p = +0), rounded
+      // to bf16 for P.V; the running sum adds the same rounded values
       uint32_t pk[32];
-      float l_chunk = 0.f;
+      float2 l2 = make_float2(0.f, 0.f);
+      const float m_sub = m_new == -INFINITY ? 0.f : m_new;  // nothing valid yet: every x is -inf
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float x0 = __uint_as_float(sv[j]), x1 = __uint_as_float(sv[j + 1]);
-        const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - m_new);
-        const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - m_new);
-        const __nv_bfloat162 pbf = __floats2bfloat162_rn(p0, p1);
-        const float2 back = __bfloat1622float2(pbf);
-        l_chunk += back.x + back.y;
+        const float2 d = __fadd2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
+                                    make_float2(-m_sub, -m_sub));
+        const __nv_bfloat162 pbf = __floats2bfloat162_rn(ex2_approx(d.x), ex2_approx(d.y));
+        l2 = __fadd2_rn(l2, __bfloat1622float2(pbf));
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&pbf);
       }
+      const float l_chunk = l2.x + l2.y;
       if (__any_sync(0xffffffffu, resc)) {
         // O is rescaled in TMEM: every earlier PV must have completed (the
         // last one, PV(i-1), completes after all the others)

@@ -205,6 +205,37 @@ def test_short_context_many_rows(cuda_device):
     check_mla(out, lse, full, sub, list(range(len(rows))))
 
 
+@pytest.mark.parametrize("B", [2, 20])  # 20 rows x 32 chunks of 64 take the 64-key kernel
+def test_attention_on_arbitrary_index_lists(cuda_device, B):
+    """dsa_sparse_mla on index lists it did not get from the selection:
+    unsorted, with repeats, -1 holes, a whole 64-slot block of -1 ahead of
+    valid slots, and one row with nothing selected (out 0, lse -inf)."""
+    from sparse_attention_04_b200 import _lib
+    k, H = 2048, 128
+    wl = dsa_inputs.custom("arb_idx", B=B, end_pos=None, end_pos_range=(2500, 6000), topk=k, H=H,
+                           out_dtype="bf16", scale=192 ** -0.5, seed=61)
+    inp = dsa_inputs.make_inputs(wl, cuda_device)
+    g = torch.Generator().manual_seed(62)
+    idx = torch.stack([torch.randint(0, E, (k,), generator=g, dtype=torch.int32) for E in inp.end_pos])
+    idx[torch.rand(B, k, generator=g) < 0.1] = -1
+    idx[:, 128:192] = -1
+    idx[:, :64] = -1  # the first chunk of every row holds nothing
+    idx[B - 1] = -1
+    idx = idx.to(cuda_device)
+    out = torch.empty(B, 1, H, 512, dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.empty(B, 1, H, dtype=torch.float32, device=cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ws = torch.empty(max(16, _lib.sparse_mla_workspace_size(B, 1, H, k)), dtype=torch.uint8, device=cuda_device)
+    _lib.sparse_mla(inp.q, inp.kv, inp.offsets, idx, B, 1, H, k, wl.scale, inp.rows, out, lse=lse, workspace=ws,
+                    status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, _lib_status(st)
+    seqs = [0, B - 1] if B == 2 else [0, 11, B - 1]
+    sub = subset(inp, seqs)
+    check_mla(out.reshape(B, H, -1)[seqs], lse.reshape(B, H)[seqs], idx[seqs], sub, list(range(len(seqs))))
+    assert torch.all(out[B - 1] == 0) and torch.all(torch.isinf(lse[B - 1]) & (lse[B - 1] < 0))
+
+
 def test_fp8_small(cuda_device):
     wl = dsa_inputs.custom("fp8s", B=2, end_pos=None, topk=128, H=128, idx_dtype="e4m3", out_dtype="bf16",
                            scale=192 ** -0.5, seed=9, end_pos_range=(1, 1))
