@@ -229,6 +229,109 @@ __device__ void radix_select_fallback(SM& sm, uint32_t* keys, int key_cap, const
   }
 }
 
+// ============================================================================
+// Short rows (ld <= kRowMaxLen: causal prefill, short decode): one CTA of
+// 256 threads per row, thread t holding the keys of positions 32t .. 32t+31
+// in registers, so the row is read once and no candidate buffer is needed.
+//   A  12-bit histogram (shared atomics) -> bin d* of the k-th largest key
+//   B  two 10-bit histograms over the keys in d* (from the registers) -> the
+//      exact k-th key tau and how many keys equal to tau are kept
+//   C  keep every key > tau and the need_eq lowest positions equal to tau
+//      (a block scan ranks the ties), then one more block scan places each
+//      thread's kept positions in the ascending output.
+// 16 KB of shared memory, so eight rows run per SM.
+constexpr int kRowThreads = 256;
+constexpr int kRowMaxLen = kRowThreads * 32;
+struct RowSmem {
+  uint32_t warp_tot[kRowThreads / 32];
+  uint32_t carry;
+  uint32_t sel_digit;
+  uint32_t sel_remaining;
+  uint32_t pad[5];
+  uint32_t hist[kBins12];
+};
+
+__global__ void __launch_bounds__(kRowThreads)
+    topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B, int T,
+                     int k, int32_t* __restrict__ indices, int32_t* status) {
+  __shared__ RowSmem sm;
+  grid_dependency_wait();  // scores come from the previous kernel
+  allow_dependents_launch();
+  const int r = blockIdx.x;
+  const int b = r / T, t = r - (r / T) * T;
+  int32_t* out = indices + (int64_t)r * k;
+  const int E = off[b + 1] - off[b];
+  if (E < T || (int64_t)E > ld || off[b] < 0) {
+    for (int j = threadIdx.x; j < k; j += kRowThreads) out[j] = -1;
+    if (threadIdx.x == 0) report(status, DSA_ERR_BAD_OFFSETS);
+    return;
+  }
+  const int L = E - T + t + 1;  // causal prefix: every valid position (<= ld <= kRowMaxLen)
+  if (L <= k) {  // every valid position is kept
+    for (int j = threadIdx.x; j < k; j += kRowThreads) out[j] = j < L ? j : -1;
+    return;
+  }
+  const float* row = scores + (int64_t)r * ld;
+  const int w = threadIdx.x;
+  uint32_t kk[32], vb = 0;
+  if (32 * w < L) {
+    load_word(row, L, w, kk, &vb);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) kk[j] = 0u;
+  }
+  for (int i = threadIdx.x; i < kBins12; i += kRowThreads) sm.hist[i] = 0;
+  __syncthreads();
+
+  // ---- A: top 12 bits
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if ((vb >> j) & 1u) atomicAdd(&sm.hist[kk[j] >> 20], 1u);
+  __syncthreads();
+  select_bin<kRowThreads>(sm, sm.hist, kBins12, (uint32_t)k);
+
+  // ---- B: bits 19..10, then 9..0, of the keys sharing the prefix so far
+  uint32_t prefix = sm.sel_digit << 20, pmask = 0xFFF00000u, remaining = sm.sel_remaining;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    for (int i = threadIdx.x; i < 1024; i += kRowThreads) sm.hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (((vb >> j) & 1u) && (kk[j] & pmask) == prefix) atomicAdd(&sm.hist[(kk[j] >> shift) & 1023u], 1u);
+    __syncthreads();
+    select_bin<kRowThreads>(sm, sm.hist, 1024, remaining);
+    prefix |= sm.sel_digit << shift;
+    pmask |= 1023u << shift;
+    remaining = sm.sel_remaining;
+  }
+  const uint32_t tau = prefix, need_eq = remaining;
+
+  // ---- C: keys above tau, plus the lowest positions equal to tau
+  uint32_t keep = 0, eq = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const bool valid = (vb >> j) & 1u;
+    keep |= (valid && kk[j] > tau ? 1u : 0u) << j;
+    eq |= (valid && kk[j] == tau ? 1u : 0u) << j;
+  }
+  uint32_t tot;
+  uint32_t rank = block_excl_scan<kRowThreads>(__popc(eq), sm, &tot);
+  while (eq && rank < need_eq) {
+    const uint32_t low = eq & (0u - eq);
+    keep |= low;
+    eq ^= low;
+    ++rank;
+  }
+  uint32_t pos = block_excl_scan<kRowThreads>(__popc(keep), sm, &tot);
+  while (keep) {
+    const int j = __ffs(keep) - 1;
+    keep &= keep - 1;
+    out[pos++] = 32 * w + j;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off,
                 int B, int T, int k, int32_t* __restrict__ indices, int32_t* status) {
@@ -788,6 +891,11 @@ int launch_topk(const TopkArgs& a, cudaStream_t stream) {
     if (DSA_TOPK_FEW_ROWS_CLUSTER == 16 && rows * 16 <= 2 * device_info().sm_count)
       return launch_cluster<16>(a, stream);
     return launch_cluster<8>(a, stream);
+  }
+  if (a.ld <= kRowMaxLen) {
+    const cudaError_t e = launch_pdl(topk_rows_kernel, dim3(rows), dim3(kRowThreads), 0, stream, a.scores, a.ld,
+                                     a.offsets, a.B, a.T, a.k, a.indices, a.status);
+    return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
   }
   static bool attr_set = false;
   if (!attr_set) {

@@ -60,3 +60,35 @@ def test_batch_of_ragged_rows(cuda_device):
     rows = [_gen(n, 100 + n) for n in (1, 31, 32, 33, 2047, 2048, 2049, 4096, 50000)]
     got, want = _run(rows, 2048)
     assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("k", [1, 4, 2047, 2048])
+def test_short_rows(cuda_device, k):
+    """Rows of at most 8192 positions (one 256-thread CTA per row, keys held
+    in registers): random rows, heavy ties, signed zeros and -inf, and ragged
+    lengths around word and block boundaries."""
+    g = torch.Generator().manual_seed(70 + k)
+    alphabet = torch.tensor([-0.0, 0.0, 1.0, -1.0, 2.5, 1e-30, -1e-30, float("-inf")])
+    rows = [_gen(n, 200 + n) for n in (2049, 2080, 4096, 5000, 8191, 8192)]
+    rows += [alphabet[torch.randint(0, 8, (7000,), generator=g)], torch.full((6000,), 0.25),
+             torch.randn(8000, generator=g).round(decimals=1), torch.randn(3000, generator=g) * 1e-20, _gen(5, 9)]
+    got, want = _run(rows, k)
+    assert torch.equal(got, want)
+
+
+def test_causal_prefill_rows(cuda_device):
+    """T = 600 query rows of one 6000-position sequence: row t keeps the top
+    k of its causal prefix of 5401 + t positions."""
+    from sparse_attention_04_b200 import _lib
+    dev = torch.device("cuda:0")
+    T, E, k = 600, 6000, 2048
+    ld = E
+    sc = torch.randn(T, ld, generator=torch.Generator().manual_seed(71))
+    sc[::7] = sc[::7].round(decimals=1)  # some rows full of ties
+    off = torch.tensor([0, E], dtype=torch.int32)
+    out = torch.empty((T, k), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _lib.topk(sc.to(dev), ld, off.to(dev), 1, T, k, out, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out.cpu(), oracle.topk(sc.double(), off, 1, T, k))
