@@ -143,7 +143,7 @@ int dsa_decode_step_launches(int B, int max_end_pos, int k, int H) {
   if (B <= 0 || max_end_pos <= 0 || k < 1 || k > DSA_MAX_TOPK || H < 1 || H > DSA_MAX_HEADS) return -1;
   int n = max_end_pos <= k ? 0 : 2;           // indexer + selection (skipped for short contexts)
   n += 1;                                      // attention
-  n += mla_num_splits(B, k, H) > 1 ? 1 : 0;    // combine of the split partials
+  n += mla_num_splits(B, k, H, max_end_pos <= k) > 1 ? 1 : 0;  // combine of the split partials
   return n;
 }
 

@@ -104,8 +104,8 @@ constexpr int kMlaWideChunk = 64;
 cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout,
                                    const MlaParams& p, unsigned grid, cudaStream_t stream);
 
-int mla_num_splits(int n_rows, int k, int H);
-int mla_chunk(int n_rows, int k);
+int mla_num_splits(int n_rows, int k, int H, bool dense);  // dense: no index list (short context)
+int mla_chunk(int n_rows, int k, bool dense);
 size_t mla_workspace_bytes(int n_rows, int H, int k);
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream);
 

@@ -576,13 +576,18 @@ __global__ void __launch_bounds__(64)
 }  // namespace
 
 // Which attention kernel a launch uses.  The 64-key kernel halves the QK
-// issue cost per key but starts its first QK only once 64 rows have landed;
-// it wins when the attention CTAs (two per row and split, one per SM) each
-// work through many chunks, i.e. when 2 * rows * 64-key chunks is at least
-// kMlaWideMinChunksPerSm times the SM count (batched decode, prefill).
+// issue cost per key, and after a selection stage it is the faster one for
+// any row count (decode 32K: 27.9 against 29.5 us per step; four 131K rows:
+// 49.0 against 52.1 us).  Its query prologue (blocks 0-5 into TMEM through
+// registers) is slower than the 32-key kernel's single TMA load, and only a
+// launch with no preceding stage to hide behind pays for it: the dense
+// short-context attention with few chunks per SM (one 2K row: 14.6 against
+// 13.9 us) keeps the 32-key kernel unless 2 * rows * 64-key chunks reaches
+// kMlaWideMinChunksPerSm times the SM count.
 constexpr int kMlaWideMinChunksPerSm = 8;
 
-int mla_chunk(int n_rows, int k) {
+int mla_chunk(int n_rows, int k, bool dense) {
+  if (!dense) return kMlaWideChunk;
   const int64_t n64 = (k + kMlaWideChunk - 1) / kMlaWideChunk;
   const int64_t sms = device_info().sm_count;
   return 2 * (int64_t)n_rows * n64 >= kMlaWideMinChunksPerSm * sms ? kMlaWideChunk : kChunk;
@@ -598,8 +603,8 @@ int mla_chunk(int n_rows, int k) {
 // little gain).
 static_assert(DSA_MAX_TOPK / 64 <= kMaxSplits, "the combine holds every split of a row in registers");
 
-int mla_num_splits(int n_rows, int k, int H) {
-  const int chunk = mla_chunk(n_rows, k);
+int mla_num_splits(int n_rows, int k, int H, bool dense) {
+  const int chunk = mla_chunk(n_rows, k, dense);
   const int n_chunks = (k + chunk - 1) / chunk;
   const int64_t sms = device_info().sm_count;
   int max_splits = n_chunks * chunk / 64;
@@ -623,9 +628,10 @@ int mla_num_splits(int n_rows, int k, int H) {
 
 namespace {
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-// Workspace: [split partials bf16][(max, sum) fp32]
+// Workspace: [split partials bf16][(max, sum) fp32], sized for whichever of
+// the index-list and dense launches splits more
 size_t mla_partials_bytes(int n_rows, int H, int k) {
-  const int ns = mla_num_splits(n_rows, k, H);
+  const int ns = std::max(mla_num_splits(n_rows, k, H, false), mla_num_splits(n_rows, k, H, true));
   if (ns <= 1) return 0;
   return align256((size_t)n_rows * ns * H * (kDV * sizeof(__nv_bfloat16) + 2 * sizeof(float)));
 }
@@ -637,8 +643,9 @@ size_t mla_workspace_bytes(int n_rows, int H, int k) {
 
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   const int n_rows = a.B * a.T;
-  const int ns = mla_num_splits(n_rows, a.k, a.H);
-  const int chunk = mla_chunk(n_rows, a.k);
+  const bool dense = a.indices == nullptr;
+  const int ns = mla_num_splits(n_rows, a.k, a.H, dense);
+  const int chunk = mla_chunk(n_rows, a.k, dense);
   const int n_chunks = (a.k + chunk - 1) / chunk;
   MlaParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
