@@ -878,24 +878,16 @@ int launch_cluster(const TopkArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-// Rows longer than kClusterMinLd positions go to the cluster kernel (16 CTAs
-// per row when there are few rows, else 8); shorter rows (prefill) take one
-// CTA each.
+// Rows longer than kClusterMinLd positions go to the cluster kernel, 8 CTAs
+// per row (16 measured slower even for a single 32K row: 28.3 against 27.3 us
+// per decode step); shorter rows (prefill) take one CTA each.
 #ifndef DSA_TOPK_CLUSTER_MIN_LD
 #define DSA_TOPK_CLUSTER_MIN_LD 8192
 #endif
 
-#ifndef DSA_TOPK_FEW_ROWS_CLUSTER
-#define DSA_TOPK_FEW_ROWS_CLUSTER 16
-#endif
-
 int launch_topk(const TopkArgs& a, cudaStream_t stream) {
   const int rows = a.B * a.T;
-  if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072) {
-    if (DSA_TOPK_FEW_ROWS_CLUSTER == 16 && rows * 16 <= 2 * device_info().sm_count)
-      return launch_cluster<16>(a, stream);
-    return launch_cluster<8>(a, stream);
-  }
+  if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072) return launch_cluster<8>(a, stream);
   if (a.ld <= kRowMaxLen) {
     const cudaError_t e = launch_pdl(topk_rows_kernel<kRowThreads>, dim3(rows), dim3(kRowThreads), 0, stream,
                                      a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
