@@ -90,6 +90,14 @@ def test_sparse_mla_argument_validation(L):
     assert f(*nan_scale) == 1
 
 
+def test_host_copy_validation(L):
+    h2d, d2h = L.lib.dsa_copy_host_to_device, L.lib.dsa_copy_device_to_host
+    assert h2d(P(A), P(A), 0, None) == 0                          # nothing to copy
+    assert h2d(P(A), P(A), 24, None) == 1                         # not a multiple of 16
+    assert h2d(None, P(A), 32, None) == 1 and d2h(P(A), None, 32, None) == 1
+    assert d2h(P(A + 8), P(A), 32, None) == 1                     # misaligned
+
+
 def test_workspace_sizes(L):
     s_off, ld, i_off, m_off = L.decode_step_workspace_layout(32, 131072, 2048, 128)
     assert s_off == 0 and ld == 131072 and i_off >= 32 * ld * 4 and m_off >= i_off + 32 * 2048 * 4
