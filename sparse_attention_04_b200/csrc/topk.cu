@@ -502,7 +502,7 @@ struct ClusterCfg {
   static constexpr int kWarps = kThreads / 32;
   static constexpr int kSliceMax = 131072 / CS;          // positions per CTA
   static constexpr int kSliceWords = kSliceMax / 32;
-  static constexpr int kPerSrc = 8192 / CS;                // candidates a CTA may send
+  static constexpr int kPerSrc = 4096 / CS;                // candidates a CTA may send (107 KB in all: two CTAs per SM)
   static_assert(kSliceWords <= kThreads, "one bitmap word per thread");
   static_assert(CS <= kWarps && CS <= 32 && 32 % CS == 0, "per-source counting and lane groups");
 };
@@ -562,7 +562,7 @@ __device__ __forceinline__ void warp_select64(const uint32_t* bins, uint32_t nee
 }
 
 template <int CS>
-__global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 1)
+__global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 2)
     topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B,
                         int T, int k, int32_t* __restrict__ indices, int32_t* status) {
   using Cfg = ClusterCfg<CS>;
