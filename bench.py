@@ -542,8 +542,19 @@ def run_prefill(dev, stream, peaks, reps=20):
         torch.cuda.synchronize()
         return ev0.elapsed_time(ev1) / 1e3 / n
 
+    def select(i):
+        x = copies[i % n_copies]
+        _lib.topk(scores[i % n_copies], ld, x.offsets, B, T, k, indices, status=status)
+
+    def attend(i):
+        x = copies[i % n_copies]
+        _lib.sparse_mla(x.q, x.kv, x.offsets, indices, B, T, H, k, wl.scale, x.rows, out, lse=lse, workspace=ws,
+                        status=status)
+
     t_idx = timed(indexer, reps)
     t_all = timed(staged, max(2, reps // 4))
+    t_sel = timed(select, reps)       # the score copies were all written above
+    t_att = timed(attend, max(2, reps // 4))
     if int(status.item()) != 0:
         raise SystemExit("prefill: device status " + _lib.status_string(int(status.item())))
     flops = prefill_indexer_flops(T, E)
@@ -552,10 +563,18 @@ def run_prefill(dev, stream, peaks, reps=20):
     except Exception:
         peak, src = 1590.0, "fallback"
     achieved = flops / t_idx / 1e12
+    # attention: 2*H*(576 + 512) flops per kept (row, key); row t keeps min(t + 1, k) keys
+    att_flops = 2 * H * (576 + 512) * sum(min(E - T + t + 1, k) for t in range(T))
+    att = att_flops / t_att / 1e12
     return {"workload": "prefill4k", "kernel": "indexer", "bound": "tensor", "us": round(t_idx * 1e6, 2),
             "flops": flops, "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "peak_source": src,
             "staged_step_us": round(t_all * 1e6, 1),
+            "stages_us": {"indexer": round(t_idx * 1e6, 1), "topk": round(t_sel * 1e6, 1),
+                          "sparse_mla": round(t_att * 1e6, 1)},
+            "attention": {"kernel": "sparse_mla", "bound": "tensor", "flops": att_flops, "achieved": round(att, 1),
+                          "peak": peak, "unit": "TFLOP/s", "frac": round(att / peak, 4),
+                          "traffic": load_traffic("prefill4k", "sparse_mla")},
             "note": "causal lower triangle only; 3 rotating input and score copies"}
 
 
