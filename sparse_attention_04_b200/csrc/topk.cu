@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // rank 0 redoes the row with the exact digit-pass fallback.
 template <int CS>
 struct ClusterCfg {
-  static constexpr int kThreads = 512;
+  static constexpr int kThreads = CS >= 8 ? 512 : 1024;
   static constexpr int kWarps = kThreads / 32;
   static constexpr int kSliceMax = 131072 / CS;          // positions per CTA
   static constexpr int kSliceWords = kSliceMax / 32;
@@ -562,13 +562,14 @@ __device__ __forceinline__ void warp_select64(const uint32_t* bins, uint32_t nee
 }
 
 template <int CS>
-__global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 2)
+__global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, ClusterCfg<CS>::kThreads == 512 ? 2 : 1)
     topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B,
                         int T, int k, int32_t* __restrict__ indices, int32_t* status) {
   using Cfg = ClusterCfg<CS>;
   constexpr int NT = Cfg::kThreads;
   constexpr uint32_t kPerSrc = Cfg::kPerSrc;
-  static_assert(NT * 8 == kBins12, "coarse sums: 8 bins per thread");
+  constexpr int BPT = kBins12 / NT, TPC = 64 / BPT;  // fine bins per thread, threads per coarse bin
+  static_assert(BPT * NT == kBins12 && TPC <= 32, "coarse sums");
   static_assert(offsetof(ClusterSmem<CS>, keys) % 16 == 0, "16-byte key stores");
   namespace cg = cooperative_groups;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -635,17 +636,18 @@ __global__ void __launch_bounds__(ClusterCfg<CS>::kThreads, 2)
   {
     uint32_t v = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) v += sm.hist[8 * threadIdx.x + j];
+    for (int j = 0; j < BPT; ++j) v += sm.hist[BPT * threadIdx.x + j];
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
-    // every lane of the 8-lane group now holds coarse sum c = tid/8; the
-    // group pushes it to all CTAs, lane i of the group to CTAs i, i+8, ...
-    const uint32_t c = threadIdx.x >> 3;
+    if (TPC > 8) v += __shfl_xor_sync(0xffffffffu, v, 8);
+    // every lane of the TPC-lane group now holds coarse sum c = tid/TPC; the
+    // group pushes it to all CTAs, lane i of the group to CTAs i, i+TPC, ...
+    const uint32_t c = threadIdx.x / TPC;
     cluster_wait();
 #pragma unroll
-    for (int i = 0; i < (CS + 7) / 8; ++i) {
-      const int q = (lane & 7) + 8 * i;
+    for (int i = 0; i < (CS + TPC - 1) / TPC; ++i) {
+      const int q = (lane % TPC) + TPC * i;
       if (q < CS) cluster.map_shared_rank(&sm, q)->all_coarse[rank][c] = v;
     }
   }
@@ -878,16 +880,19 @@ int launch_cluster(const TopkArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-// Rows longer than kClusterMinLd positions go to the cluster kernel, 8 CTAs
-// per row (16 measured slower even for a single 32K row: 28.3 against 27.3 us
-// per decode step); shorter rows (prefill) take one CTA each.
+// Rows longer than kClusterMinLd positions go to the cluster kernel: 8 CTAs
+// of 512 threads per row for up to three rows (a single 32K row: 27.3 us per
+// decode step against 28.3 with 16 CTAs and 27.9 with 4), 4 CTAs of 1024
+// threads per row from four rows on (four 131K rows: 47.0 against 47.7 us;
+// 32 rows: 178 against 182 us).  Shorter rows (prefill) take one CTA each.
 #ifndef DSA_TOPK_CLUSTER_MIN_LD
 #define DSA_TOPK_CLUSTER_MIN_LD 8192
 #endif
 
 int launch_topk(const TopkArgs& a, cudaStream_t stream) {
   const int rows = a.B * a.T;
-  if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072) return launch_cluster<8>(a, stream);
+  if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072)
+    return rows >= 4 ? launch_cluster<4>(a, stream) : launch_cluster<8>(a, stream);
   if (a.ld <= kRowMaxLen) {
     const cudaError_t e = launch_pdl(topk_rows_kernel<kRowThreads>, dim3(rows), dim3(kRowThreads), 0, stream,
                                      a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
