@@ -236,6 +236,16 @@ def test_attention_on_arbitrary_index_lists(cuda_device, B):
     assert torch.all(out[B - 1] == 0) and torch.all(torch.isinf(lse[B - 1]) & (lse[B - 1] < 0))
 
 
+def test_decode_mixed_lengths_long_pitch(cuda_device):
+    """One decode step over rows of 5 to 70000 positions (score pitch above
+    8192, so the selection runs as 4-CTA clusters): rows that keep every
+    position sit beside rows that select, and the attention's splits of the
+    short rows hold few or no chunks."""
+    wl = dsa_inputs.custom("mixed", B=5, end_pos=None, topk=2048, H=16, out_dtype="bf16", scale=192 ** -0.5,
+                           seed=63, end_pos_range=(1, 1))
+    run_and_check(wl, cuda_device, end_pos=[5, 2000, 9000, 40000, 70000])
+
+
 def test_fp8_small(cuda_device):
     wl = dsa_inputs.custom("fp8s", B=2, end_pos=None, topk=128, H=128, idx_dtype="e4m3", out_dtype="bf16",
                            scale=192 ** -0.5, seed=9, end_pos_range=(1, 1))
