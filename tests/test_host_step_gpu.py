@@ -77,3 +77,35 @@ def test_host_step_matches_device_path_and_oracle(cuda_device, idx_dtype, eps, k
             idx = hs.step.indices.cpu()
         sub = Inputs(wl, list(eps), inp.offsets.cpu(), None, None, None, None, hs.host_q.clone(), inp.kv.cpu())
         check_mla(out.reshape(B, H, -1), hs.step.lse.reshape(B, H), idx, sub, list(range(B)))
+
+
+def test_host_step_in_a_cuda_graph(cuda_device):
+    """Captured once, replayed with the host inputs refilled between
+    replays: each replay's output matches an eager host-fed step on the same
+    inputs and caches."""
+    from sparse_attention_04_b200 import api
+    B, H, k = 2, 16, 512
+    eps = [9000, 3000]
+    wl = dsa_inputs.custom("host_graph", B=B, end_pos=None, topk=k, H=H, out_dtype="bf16", seed=91,
+                           end_pos_range=(1, 1))
+    inp = dsa_inputs.make_inputs(wl, cuda_device, end_pos=eps)
+    hs = api.HostDecodeStep(B, max(eps), k, H, "bf16", torch.bfloat16, cuda_device)
+    ref_hs = api.HostDecodeStep(B, max(eps), k, H, "bf16", torch.bfloat16, cuda_device)
+    kv2, k2 = inp.kv.clone(), inp.k_idx.clone()
+    stream = torch.cuda.Stream(cuda_device)
+    _fill_host(hs, B, H, 100)
+    with torch.cuda.stream(stream):
+        hs(inp.k_idx, inp.k_scale, inp.kv, inp.offsets, inp.rows, wl.scale)  # warm-up, outside the graph
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        hs(inp.k_idx, inp.k_scale, inp.kv, inp.offsets, inp.rows, wl.scale)
+    for seed in (101, 102, 103):
+        _fill_host(hs, B, H, seed)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(hs.step.status.item()) == 0
+        _fill_host(ref_hs, B, H, seed)
+        ref = ref_hs(k2, None, kv2, inp.offsets, inp.rows, wl.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(hs.host_out.view(torch.int16), ref.view(torch.int16))
