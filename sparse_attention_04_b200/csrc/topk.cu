@@ -143,6 +143,35 @@ __device__ __forceinline__ void load_word(const float* __restrict__ row, int L, 
   }
 }
 
+// Keys of positions KPT*w .. KPT*w + KPT-1 (KPT = 16 or 32); bits of
+// *valid_bits mark positions < L.
+template <int KPT>
+__device__ __forceinline__ void load_keys(const float* __restrict__ row, int L, int w, uint32_t (&kk)[KPT],
+                                          uint32_t* valid_bits) {
+  const int s0 = KPT * w;
+  if (s0 + KPT <= L) {
+    const float4* p = reinterpret_cast<const float4*>(row + s0);
+#pragma unroll
+    for (int j = 0; j < KPT / 4; ++j) {
+      const float4 v = __ldg(p + j);
+      kk[4 * j + 0] = float_order_key(v.x);
+      kk[4 * j + 1] = float_order_key(v.y);
+      kk[4 * j + 2] = float_order_key(v.z);
+      kk[4 * j + 3] = float_order_key(v.w);
+    }
+    *valid_bits = KPT == 32 ? 0xffffffffu : (1u << KPT) - 1u;
+  } else {
+    uint32_t vb = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const bool ok = s0 + j < L;
+      kk[j] = ok ? load_key(row, s0 + j) : 0u;
+      vb |= (ok ? 1u : 0u) << j;
+    }
+    *valid_bits = vb;
+  }
+}
+
 // Writes the positions of the set bits of bitmap[0 .. n_words) ascending into out.
 template <class SM>
 __device__ __forceinline__ void emit_bitmap(SM& sm, const uint32_t* bitmap, int n_words, int32_t* out) {
@@ -231,8 +260,9 @@ __device__ void radix_select_fallback(SM& sm, uint32_t* keys, int key_cap, const
 
 // ============================================================================
 // Short rows (ld <= kRowMaxLen: causal prefill, short decode): one CTA of
-// 256 threads per row, thread t holding the keys of positions 32t .. 32t+31
-// in registers, so the row is read once and no candidate buffer is needed.
+// 256 threads per row, thread t holding the keys of positions KPT*t ..
+// KPT*t + KPT-1 in registers (KPT = 16 for rows of up to 4096 positions, else
+// 32), so the row is read once and no candidate buffer is needed.
 //   A  12-bit histogram (shared atomics) -> bin d* of the k-th largest key
 //   B  two 10-bit histograms over the keys in d* (from the registers) -> the
 //      exact k-th key tau and how many keys equal to tau are kept
@@ -254,7 +284,7 @@ struct RowSmem {
   uint32_t hist[kBins12];
 };
 
-template <int NT>
+template <int NT, int KPT>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 4 : 1)  // four rows per SM at 256 threads (64 registers)
     topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ off, int B, int T,
                      int k, int32_t* __restrict__ indices, int32_t* status) {
@@ -277,19 +307,19 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 4 : 1)  // four rows per SM at
   }
   const float* row = scores + (int64_t)r * ld;
   const int w = threadIdx.x;
-  uint32_t kk[32], vb = 0;
-  if (32 * w < L) {
-    load_word(row, L, w, kk, &vb);
+  uint32_t kk[KPT], vb = 0;  // the keys of positions KPT*w .. KPT*w + KPT-1
+  if (KPT * w < L) {
+    load_keys<KPT>(row, L, w, kk, &vb);
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) kk[j] = 0u;
+    for (int j = 0; j < KPT; ++j) kk[j] = 0u;
   }
   for (int i = threadIdx.x; i < kBins12; i += NT) sm.hist[i] = 0;
   __syncthreads();
 
   // ---- A: top 12 bits
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
+  for (int j = 0; j < KPT; ++j)
     if ((vb >> j) & 1u) atomicAdd(&sm.hist[kk[j] >> 20], 1u);
   __syncthreads();
   select_bin<NT>(sm, sm.hist, kBins12, (uint32_t)k);
@@ -302,7 +332,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 4 : 1)  // four rows per SM at
     for (int i = threadIdx.x; i < 1024; i += NT) sm.hist[i] = 0;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
+    for (int j = 0; j < KPT; ++j)
       if (((vb >> j) & 1u) && (kk[j] & pmask) == prefix) atomicAdd(&sm.hist[(kk[j] >> shift) & 1023u], 1u);
     __syncthreads();
     select_bin<NT>(sm, sm.hist, 1024, remaining);
@@ -315,7 +345,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 4 : 1)  // four rows per SM at
   // ---- C: keys above tau, plus the lowest positions equal to tau
   uint32_t keep = 0, eq = 0;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < KPT; ++j) {
     const bool valid = (vb >> j) & 1u;
     keep |= (valid && kk[j] > tau ? 1u : 0u) << j;
     eq |= (valid && kk[j] == tau ? 1u : 0u) << j;
@@ -332,7 +362,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 4 : 1)  // four rows per SM at
   while (keep) {
     const int j = __ffs(keep) - 1;
     keep &= keep - 1;
-    out[pos++] = 32 * w + j;
+    out[pos++] = KPT * w + j;
   }
 }
 
@@ -894,7 +924,10 @@ int launch_topk(const TopkArgs& a, cudaStream_t stream) {
   if (a.ld > DSA_TOPK_CLUSTER_MIN_LD && a.ld <= 131072)
     return rows >= 4 ? launch_cluster<4>(a, stream) : launch_cluster<8>(a, stream);
   if (a.ld <= kRowMaxLen) {
-    const cudaError_t e = launch_pdl(topk_rows_kernel<kRowThreads>, dim3(rows), dim3(kRowThreads), 0, stream,
+    // rows of up to 4096 positions: 16 keys per thread, so every thread has work
+    const cudaError_t e = launch_pdl(a.ld <= kRowThreads * 16 ? topk_rows_kernel<kRowThreads, 16>
+                                                              : topk_rows_kernel<kRowThreads, 32>,
+                                     dim3(rows), dim3(kRowThreads), 0, stream,
                                      a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
     return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
   }

@@ -92,3 +92,17 @@ def test_causal_prefill_rows(cuda_device):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert torch.equal(out.cpu(), oracle.topk(sc.double(), off, 1, T, k))
+
+
+@pytest.mark.parametrize("k", [1, 37, 2048])
+def test_short_rows_16_keys_per_thread(cuda_device, k):
+    """Rows of at most 4096 positions take 16 keys per thread: random rows,
+    heavy ties, signed zeros and -inf, ragged lengths around the 16-key
+    groups."""
+    g = torch.Generator().manual_seed(90 + k)
+    alphabet = torch.tensor([-0.0, 0.0, 1.0, -1.0, 2.5, 1e-30, -1e-30, float("-inf")])
+    rows = [_gen(n, 300 + n) for n in (2049, 2065, 3000, 4095, 4096)]
+    rows += [alphabet[torch.randint(0, 8, (4000,), generator=g)], torch.full((3500,), -0.5),
+             torch.randn(4096, generator=g).round(decimals=1), _gen(17, 3)]
+    got, want = _run(rows, k)
+    assert torch.equal(got, want)
