@@ -108,7 +108,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!p.early_inputs) grid_dependency_wait();  // q and the offsets may come from the previous kernel
   const int v = blockIdx.x & 1;
   const int sp = (blockIdx.x >> 1) % p.n_splits;
-  const int r = (blockIdx.x >> 1) / p.n_splits;
+  // rows in reverse launch order: a causal prefill's late rows keep the most
+  // keys, and launching them first leaves the short rows to fill the last
+  // wave (prefill 4K attention 4.27 -> 4.20 ms)
+  const int r = (int)(gridDim.x / (2 * p.n_splits)) - 1 - (int)((blockIdx.x >> 1) / p.n_splits);
   const int b = r / p.T;
   const int32_t base_row = p.off[b];
   const int E = p.off[b + 1] - base_row;
