@@ -114,15 +114,20 @@ class ClockSampler:
                 pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
             mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
 
+            def sample():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                         int(get_reasons(h))))
+                except Exception:
+                    pass
+
             def loop():
                 while not self.stop_flag:
-                    try:
-                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
-                                             int(get_reasons(h))))
-                    except Exception:
-                        pass
+                    sample()
                     time.sleep(self.period)
 
+            self._sample = sample
+            sample()  # one sample as the region starts, however short it is
             self.thread = threading.Thread(target=loop, daemon=True)
             self.thread.start()
             return
@@ -142,6 +147,7 @@ class ClockSampler:
         if self.thread is not None:
             self.stop_flag = True
             self.thread.join(timeout=2)
+            self._sample()  # and one as it ends
             sm = [x[0] for x in self.samples]
             reasons = sorted({name for _, _, m in self.samples for bit, name in self.REASONS.items() if m & bit})
             return {"sm_mhz": statistics.median(sm) if sm else None,
@@ -263,22 +269,30 @@ def time_oracle(wl, inp_cpu, n_steps, seconds_per_step_budget):
 
 # ---------------------------------------------------------------- native arm
 
-def run_native(args, rank, world, local):
+def load_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {}
+
+
+def hbm_peak_of(peaks):
+    try:
+        return float(peaks["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def measure_decode(args, wl, dev, stream, world, K, W, peaks, with_e2e):
+    """Times exactly K decode steps of workload `wl` (CUDA graphs replayed on
+    `stream`, every step on its own cold cache copy), then the stages one by
+    one.  Returns a dict with the step rate, the per-stage times and
+    rooflines, the clock record of the timed region and (with_e2e) the
+    end-to-end leg."""
     import torch
     from sparse_attention_04_b200 import _lib, api
     from sparse_attention_04_b200 import inputs as I
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    wl = I.WORKLOADS[args.workload]
-    if wl.T != 1:
-        run_prefill_only(args, rank, world, dev)
-        return
     base = I.make_inputs(wl, dev)
     E = base.end_pos
     max_e = max(E)
@@ -303,11 +317,9 @@ def run_native(args, rank, world, local):
     one_step(0)
     torch.cuda.synchronize()
     if int(step.status.item()) != 0:
-        raise SystemExit("device status " + _lib.status_string(int(step.status.item())))
+        raise SystemExit(f"{wl.name}: device status " + _lib.status_string(int(step.status.item())))
 
-    K, W = args.steps, args.warmup
     G = min(K, args.graph_steps)
-    stream = torch.cuda.Stream(dev)
 
     def capture(n, start):
         g = torch.cuda.CUDAGraph()
@@ -321,10 +333,15 @@ def run_native(args, rank, world, local):
     graph_warm = capture(min(W, G), 0) if W > 0 else None
     launches_per_step = _lib.decode_step_launches(wl.B, max_e, wl.topk, wl.H)
 
-    # ---- warm-up (untimed)
+    # ---- warm-up (untimed): W steps, then one replay of every graph the
+    # timed region replays, so that no graph's first launch (its upload to
+    # the device) falls inside the events
     for _ in range(max(1, W // max(1, min(W, G)))):
         if graph_warm is not None:
             graph_warm.replay()
+    graph_main.replay()
+    if graph_rem is not None:
+        graph_rem.replay()
     torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps (clocks sampled throughout)
@@ -368,9 +385,12 @@ def run_native(args, rank, world, local):
             _lib.sparse_mla(x.q, x.kv, x.offsets, step.indices, wl.B, 1, wl.H, wl.topk, wl.scale, rows,
                             step.out, lse=step.lse, workspace=ws_mla, status=step.status)
             evs[i][3].record()
+    clocks_st = ClockSampler(dev)
+    clocks_st.start()
     g_prof.replay()
     g_prof.replay()
     torch.cuda.synchronize()
+    clk_st = clocks_st.stop()
     names = ["indexer", "topk", "sparse_mla"]
     stage_s = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_prof)) / n_prof / 1e3
                for j, n in enumerate(names)}
@@ -380,49 +400,105 @@ def run_native(args, rank, world, local):
         names = ["sparse_mla"]
         stage_s = {"sparse_mla": ms_per_step / 1e3}
     dominant = max(stage_s, key=stage_s.get)
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
-    except Exception:
-        hbm_peak, peak_src = 6650.0, "fallback"
+    hbm_peak, peak_src = hbm_peak_of(peaks)
     achieved = sb[dominant] / stage_s[dominant] / 1e9
-    traffic = load_traffic(args.workload, dominant)
+    traffic = load_traffic(wl.name, dominant)
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "peak_source": peak_src,
                 "stage_us": {n: round(v * 1e6, 3) for n, v in stage_s.items()},
                 "stage_frac": {n: round(sb[n] / stage_s[n] / 1e9 / hbm_peak, 4) for n in names},
-                "step_frac": round(sb["step"] * (value / world) / 1e9 / hbm_peak, 4)}
+                "step_frac": round(sb["step"] * (value / world) / 1e9 / hbm_peak, 4),
+                "stage_clocks": clk_st}
+    res = {"value": value, "ms_per_step": ms_per_step, "roofline": roofline, "clocks": clk, "end_pos": E,
+           "n_copies": n_copies, "bytes_per_step": sb["step"], "launches": launches_per_step * K,
+           "indexer_keys_per_s": round(sum(E) / stage_s["indexer"], 1) if "indexer" in stage_s else None}
+    if with_e2e:
+        res["e2e"] = run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world)
+    del g_prof, graph_main, graph_rem, graph_warm, copies
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
-    # ---- end to end: host buffers in, host result out, through the C ABI
-    e2e = run_e2e(args, wl, copies, n_copies, step, stream, dev, K, G, world)
-    del copies
-    prefill = None if args.no_prefill else run_prefill(dev, stream, peaks)
-    prestage = None if args.no_prefill else run_prestage(dev, stream, peaks)
 
-    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
+def decode_config(wl, end_pos, world):
+    """The `config` object of a decode line (both arms print the same one)."""
+    E = end_pos
+    return {"workload": wl.name, "B": wl.B, "end_pos": E if len(E) <= 4 else {"min": min(E), "max": max(E),
+                                                                               "sum": sum(E)},
+            "topk": wl.topk, "heads": wl.H, "indexer": f"64x128 {wl.idx_dtype}",
+            "parallelism": f"replicas x{world}",
+            "l2": "cold: every step reads its own copy of the caches, copies rotating over > 3x L2",
+            "algorithmic_bytes_per_step": stage_bytes(wl, E)["step"]}
+
+
+def run_native(args, rank, world, local):
+    import torch
+    from sparse_attention_04_b200 import inputs as I
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = I.WORKLOADS[args.workload]
+    if wl.T != 1:
+        run_prefill_only(args, rank, world, dev)
+        return
+    peaks = load_peaks()
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.Stream(dev)
+    main = measure_decode(args, wl, dev, stream, world, K, W, peaks, with_e2e=True)
+    E = main["end_pos"]
+
+    # the other decode workloads, same measurement (no end-to-end leg)
+    extra = {}
+    if not args.no_extra and args.workload == "decode32k":
+        for name in ("batched", "fp8"):
+            r = measure_decode(args, I.WORKLOADS[name], dev, stream, world, K, W, peaks, with_e2e=False)
+            ewl = I.WORKLOADS[name]
+            extra[name] = {"workload": name, "B": ewl.B, "indexer": f"64x128 {ewl.idx_dtype}",
+                           "end_pos": r["end_pos"] if len(r["end_pos"]) <= 4 else
+                           {"min": min(r["end_pos"]), "max": max(r["end_pos"]), "sum": sum(r["end_pos"])},
+                           "steps_per_s": round(r["value"], 2), "ms_per_step": round(r["ms_per_step"], 6),
+                           "algorithmic_bytes_per_step": r["bytes_per_step"],
+                           "step_frac": r["roofline"]["step_frac"], "stage_us": r["roofline"]["stage_us"],
+                           "indexer_keys_per_s": r["indexer_keys_per_s"], "roofline": r["roofline"],
+                           "clocks": r["clocks"], "l2": f"cold: {r['n_copies']} rotating cache copies",
+                           "gpu_launches": r["launches"]}
+
+    prefill = prestage = None
+    if not args.no_prefill:
+        clocks = ClockSampler(dev)
+        clocks.start()
+        prefill = run_prefill(dev, stream, peaks)
+        prefill["clocks"] = clocks.stop()
+        clocks = ClockSampler(dev)
+        clocks.start()
+        prestage = run_prestage(dev, stream, peaks)
+        prestage["clocks"] = clocks.stop()
+
+    line = {"metric": METRIC, "value": round(main["value"], 2), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(main["ms_per_step"], 6), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if wl.idx_dtype == "bf16" else "e4m3+bf16",
             "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
-            "config": {"workload": args.workload, "B": wl.B, "end_pos": E if len(E) <= 4 else
-                       {"min": min(E), "max": max(E), "sum": sum(E)}, "topk": wl.topk, "heads": wl.H,
-                       "indexer": f"64x128 {wl.idx_dtype}", "parallelism": f"replicas x{world}",
-                       "l2": f"cold: {n_copies} rotating cache copies (> 3x L2)",
-                       "algorithmic_bytes_per_step": sb["step"]},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * K, "clocks": clk}
+            "config": decode_config(wl, E, world),
+            "cache_copies": main["n_copies"], "roofline": main["roofline"], "e2e": main["e2e"], "gpu_launches": main["launches"],
+            "clocks": main["clocks"], "indexer_keys_per_s": main["indexer_keys_per_s"]}
+    line.update(extra)
     if prefill is not None:
         line["prefill_indexer"] = prefill
     if prestage is not None:
         line["indexer_prestage"] = prestage
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = base.to("cpu")
-        v, cores, text = time_oracle(wl, cpu, n_steps=3, seconds_per_step_budget=args.cpu_seconds / 3)
+        base = I.make_inputs(wl, "cpu")
+        v, cores, text = time_oracle(wl, base, n_steps=3, seconds_per_step_budget=args.cpu_seconds / 3)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": text}
     if world > 1:
         import torch.distributed as dist
-        del g_prof, graph_main, graph_rem, graph_warm
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
@@ -677,8 +753,9 @@ def run_reference(args, rank, world):
     inp = I.make_inputs(wl, "cpu")
     budget = max(0.002, args.reference_seconds / max(1, args.steps + args.warmup))
     import oracle
-    sample, frac = oracle_step_inputs(wl, inp, 1e6)
-    # calibrate, then size the per-step sample to the budget
+    # calibrate the multiply-add rate on a sample large enough that fixed
+    # costs do not dominate, then run whole steps when they fit the budget
+    sample, frac = oracle_step_inputs(wl, inp, 2e8)
     t0 = time.perf_counter()
     oracle.decode_step(sample)
     rate = oracle_work(sample.wl, sample.end_pos) / max(time.perf_counter() - t0, 1e-6)
@@ -695,8 +772,8 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded N(0,1))", "config": {"workload": args.workload, "B": wl.B,
-                                                           "topk": wl.topk, "heads": wl.H},
+            "data": "synthetic (seeded N(0,1))", "config": decode_config(wl, inp.end_pos, world),
+            "same_config": frac >= 1.0,
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": text},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -715,6 +792,7 @@ def main():
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the causal 4K prefill indexer measurement")
+    ap.add_argument("--no-extra", action="store_true", help="skip the batched and fp8 decode measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

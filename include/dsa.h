@@ -233,6 +233,24 @@ int dsa_sparse_mla_noalloc(const void* q, const void* kv, const int32_t* offsets
                            int32_t* dev_status, void* stream);
 
 /*
+ * Test hook for the device-side timeout path.  The paper has no counterpart:
+ * it exists so that a test can make a pipeline wait run out on purpose
+ * without faulting or hanging the GPU.
+ *
+ * The next n_launches attention-stage launches in this process (from
+ * dsa_sparse_mla, dsa_decode_step or dsa_sparse_mla_noalloc) initialise their
+ * query barrier with one expected arrival more than will ever come, and limit
+ * every pipeline wait to wait_limit_ns (1 ms to 1 s).  The wait runs out; the
+ * kernel stops its pipeline, waits (bounded) for its own copies and tensor
+ * core work, releases its tensor memory and writes DSA_ERR_TIMEOUT into
+ * *dev_status.  The output of such a launch is undefined; the launches after
+ * it run normally.  n_launches = 0 cancels.  Returns DSA_ERR_INVALID_ARG for
+ * a negative count or a limit outside the range.  Launches captured in a
+ * CUDA graph keep the setting they were captured with.
+ */
+int dsa_debug_stall_attention(int n_launches, uint64_t wait_limit_ns);
+
+/*
  * Where, inside a decode-step workspace, the step leaves its intermediates
  * (byte offsets; the scores pitch is returned in *ld_scores).  For tests and
  * tools that want to look at stage outputs; the layout may change between

@@ -24,7 +24,7 @@ EXPORTS = ("dsa_status_string", "dsa_version", "dsa_indexer_scores", "dsa_topk",
            "dsa_sparse_mla_workspace_size", "dsa_sparse_mla", "dsa_decode_step_workspace_size",
            "dsa_decode_step", "dsa_decode_step_workspace_layout", "dsa_sparse_mla_noalloc",
            "dsa_decode_step_launches", "dsa_cache_append", "dsa_quantize_queries", "dsa_indexer_prestage",
-           "dsa_copy_host_to_device", "dsa_copy_device_to_host")
+           "dsa_copy_host_to_device", "dsa_copy_device_to_host", "dsa_debug_stall_attention")
 
 
 class DSAError(RuntimeError):
@@ -55,6 +55,7 @@ def _load():
         "dsa_indexer_prestage": ([P, P, I, I, P, P, I, P, P, P], I),
         "dsa_copy_host_to_device": ([P, P, SZ, P], I),
         "dsa_copy_device_to_host": ([P, P, SZ, P], I),
+        "dsa_debug_stall_attention": ([I, ctypes.c_uint64], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -182,6 +183,12 @@ def copy_device_to_host(dst_host, src, stream=None):
     if dst_host.numel() * dst_host.element_size() != n:
         raise DSAError(1, "copy_device_to_host: sizes differ")
     _check(lib.dsa_copy_device_to_host(_host_p(dst_host), _p(src), n, _stream(stream)), "dsa_copy_device_to_host")
+
+
+def debug_stall_attention(n_launches: int, wait_limit_ns: int = 0):
+    """dsa_debug_stall_attention: the next n_launches attention launches take
+    their timeout path after wait_limit_ns (a test hook)."""
+    _check(lib.dsa_debug_stall_attention(n_launches, wait_limit_ns), "dsa_debug_stall_attention")
 
 
 def decode_step_launches(B, max_end_pos, k, H) -> int:

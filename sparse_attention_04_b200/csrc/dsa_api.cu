@@ -98,10 +98,12 @@ size_t dsa_sparse_mla_workspace_size(int B, int T, int H, int k) {
 namespace {
 int sparse_mla_call(const void* q, const void* kv, const int32_t* offsets, const int32_t* indices, int B, int T,
                     int H, int k, float scale, int64_t kv_rows, void* out, int out_dtype, float* lse,
-                    void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool early_inputs) {
+                    void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream, bool early_inputs,
+                    bool dense = false) {
   if (int rc = check_rows(B, T)) return rc;
-  // a NULL index list is the decode step's dense path (every prefix <= k)
-  if (!q || !kv || !offsets || (!indices && !early_inputs) || !out) return DSA_ERR_INVALID_ARG;
+  // dense: no index list, the decode step's short-context path (every prefix <= k)
+  if (!q || !kv || !offsets || (!indices && !dense) || !out) return DSA_ERR_INVALID_ARG;
+  if (dense) indices = nullptr;
   if (H < 1 || k < 1 || k > DSA_MAX_TOPK) return DSA_ERR_INVALID_ARG;
   if (H > DSA_MAX_HEADS) return DSA_ERR_UNSUPPORTED;
   if (out_dtype != DSA_BF16 && out_dtype != DSA_F32) return DSA_ERR_INVALID_ARG;
@@ -178,8 +180,12 @@ int dsa_decode_step(const void* q_idx, const float* w, const void* k_idx, const 
     // workspace are left unwritten.
     if (!q_idx || !w || !k_idx || !offsets) return DSA_ERR_INVALID_ARG;
     if (idx_dtype != DSA_BF16 && idx_dtype != DSA_E4M3) return DSA_ERR_INVALID_ARG;
+    // The attention is this call's first kernel here: nothing launched by
+    // the library has waited for the work before it in the stream (a copy
+    // kernel that may still be writing q, say), so it reads its inputs only
+    // after its own dependency wait.
     return sparse_mla_call(q, kv, offsets, nullptr, B, 1, H, k, scale, kv_rows, out, out_dtype, lse, ws + m_off,
-                           ws_bytes - m_off, dev_status, stream, true);
+                           ws_bytes - m_off, dev_status, stream, /*early_inputs=*/false, /*dense=*/true);
   }
   int rc = dsa_indexer_scores(q_idx, w, k_idx, k_scale, idx_dtype, offsets, B, 1, kv_rows, scores,
                               ld, dev_status, stream);

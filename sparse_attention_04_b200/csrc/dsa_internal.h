@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "../../include/dsa.h"
 
 namespace dsa {
@@ -29,6 +31,31 @@ struct DeviceInfo {
   int max_smem_optin;
 };
 const DeviceInfo& device_info();
+
+// Runs `set` (kernel attribute calls) once per device, under a lock.  CUDA
+// keeps a kernel's attributes (dynamic shared-memory limit, cluster size
+// permission) per device context, so a process that calls the library on
+// several GPUs must set them on each before its first launch there.
+class PerDeviceOnce {
+ public:
+  template <class Fn>
+  cudaError_t run(Fn&& set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (cached && done_[dev]) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess && cached) done_[dev] = true;
+    return e;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu_;
+  bool done_[kMaxDevices] = {};
+};
 
 // ---- stage 1: indexer ------------------------------------------------------
 struct IndexerArgs {
@@ -96,7 +123,14 @@ struct MlaParams {
   int32_t* status;
   int early_inputs;  // q and offsets may be read before the dependency wait
   int dense;         // no index list: row r attends to its whole causal prefix
+  // Test hook (dsa_debug_stall_attention): 1 makes the query barrier expect
+  // one arrival more than will ever come, so its wait runs out and the
+  // kernel takes its timeout path.  0 in normal use.
+  int debug_stall;
+  uint64_t wait_limit_ns;  // limit of every pipeline wait (kWaitLimitNs in normal use)
 };
+// Settings of the next attention launch: normal, or stalled by the test hook.
+void take_attention_debug(MlaParams& p);
 
 // The attention kernel for long index lists (sparse_mla_wide.cu): 64-key
 // chunks, grid of 2 CTAs per (row, split) as the 32-key kernel.

@@ -534,13 +534,10 @@ int launch_cfg(const IndexerArgs& a, cudaStream_t stream) {
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   auto kern = indexer_kernel<NQ, FP8>;
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;  // per template instance
+  if (attr.run([&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES); }) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   const int grid = device_info().sm_count * C::CTAS_PER_SM;
   const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, tq, tk,
                                    a.w, a.k_scale, a.offsets, a.B, a.T, a.kv_rows, a.scores, a.ld,

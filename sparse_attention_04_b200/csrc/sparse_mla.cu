@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "dsa_internal.h"
 #include "sm100.cuh"
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x < kMaxChunks) misc->vmask[threadIdx.x] = 0u;
   if (warp == 8) {
     if (lane == 0) {
-      mbar_init(q_full, 1);
+      mbar_init(q_full, 1 + p.debug_stall);  // + the test hook's missing arrival
       for (int i = 0; i < 2; ++i) {
         mbar_init(kv_full(i), 64);  // one arrival per gather thread
         mbar_init(kv_empty(i), 1);
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the load of chunk j+2 without waiting for chunk j+1 to land.
     if (lane == 0) {
       int n_qk = 0, n_pv = 0;
-      bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
+      bool ok = mbar_wait(q_full, 0, abort, p.wait_limit_ns);
       // Descriptors differ only in the start-address field (address >> 4 in
       // the low 14 bits, no carry below 256 KiB): built once, offset per MMA.
       const uint64_t qk_a0 = smem_desc(sbase + kOffQ, 16, 1024, kSwizzle128B);
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!progressed && (++spins & 63u) == 0) {  // bounded, like every other wait here
           if (*abort) ok = false;
-          else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          else if (globaltimer_ns() - t0 > p.wait_limit_ns) {
             *abort = 1;
             ok = false;
           }
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const __nv_bfloat16* kv = p.kv;
     for (int i = grp; i < n_my; i += 2) {
       const int st = i & 1;
-      if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, kWaitLimitNs)) break;
+      if (!mbar_wait(kv_empty(st), ((i >> 1) & 1) ^ 1, abort, p.wait_limit_ns)) break;
       int32_t my_id = -1;
       if (lane < 16) {
         const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < n_my; ++i) {
       const int st = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(st), (i >> 1) & 1, abort, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(st), (i >> 1) & 1, abort, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[32];
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float l_chunk = l2.x + l2.y;
       if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort, kWaitLimitNs));
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort, p.wait_limit_ns));
         if (!ok) break;
         tc_fence_after();
       }
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_my - 1) & 1, abort, kWaitLimitNs));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n_my - 1) & 1, abort, p.wait_limit_ns));
     // Every MMA has completed, so the query tile's shared memory is free: the
     // 128 x 256 result is staged there as 128-byte-swizzled boxes of 32 fp32
     // (or 64 bf16) columns, one thread per head row, and written by a few
@@ -641,6 +642,23 @@ size_t mla_workspace_bytes(int n_rows, int H, int k) {
   return mla_partials_bytes(n_rows, H, k);
 }
 
+namespace {
+std::atomic<int> g_stall_left{0};
+std::atomic<uint64_t> g_stall_limit_ns{0};
+}  // namespace
+
+void take_attention_debug(MlaParams& p) {
+  p.debug_stall = 0;
+  p.wait_limit_ns = kWaitLimitNs;
+  int left = g_stall_left.load();
+  while (left > 0 && !g_stall_left.compare_exchange_weak(left, left - 1)) {
+  }
+  if (left > 0) {
+    p.debug_stall = 1;
+    p.wait_limit_ns = g_stall_limit_ns.load();
+  }
+}
+
 int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   const int n_rows = a.B * a.T;
   const bool dense = a.indices == nullptr;
@@ -667,6 +685,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.early_inputs = a.early_inputs ? 1 : 0;
   p.dense = a.indices == nullptr ? 1 : 0;
+  take_attention_debug(p);
   if (ns > 1) {
     p.ws_o = reinterpret_cast<__nv_bfloat16*>(a.workspace);  // partials first
     p.ws_ml = reinterpret_cast<float*>(p.ws_o + (size_t)n_rows * ns * a.H * kDV);
@@ -687,13 +706,10 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     tm_ok = make_tmap_2d(&tout, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kDV, (uint64_t)n_rows * a.H, kDV * 4, 32,
                          (uint32_t)a.H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!tm_ok) return DSA_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  if (attr.run([] { return cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                kSmemBytes); }) != cudaSuccess)
+    return DSA_ERR_CUDA;
   const int64_t grid = (int64_t)n_rows * ns * 2;
   const cudaError_t e =
       chunk == kMlaWideChunk
@@ -710,3 +726,11 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace dsa
+
+extern "C" int dsa_debug_stall_attention(int n_launches, uint64_t wait_limit_ns) {
+  if (n_launches < 0) return DSA_ERR_INVALID_ARG;
+  if (n_launches > 0 && (wait_limit_ns < 1000000ull || wait_limit_ns > 1000000000ull)) return DSA_ERR_INVALID_ARG;
+  dsa::g_stall_limit_ns.store(wait_limit_ns);
+  dsa::g_stall_left.store(n_launches);
+  return DSA_OK;
+}

@@ -3,11 +3,11 @@
 //
 // "DeepSeek-V3.2-Exp - Apply sparse mask", MQA decode listing (the same
 // computation as sparse_mla.cu; see there for the formulas).  This kernel
-// serves launches whose attention CTAs each work through many chunks
-// (batched decode, causal prefill): there the issue cost of QK dominates,
-// and 64-key chunks halve it per key.  Launches with a few chunks per CTA
-// (a single long row) keep the 32-key kernel, whose first QK starts after
-// half as many rows have landed.
+// serves every launch with an index list (after a selection stage: decode
+// at any batch, causal prefill), where 64-key chunks halve the QK issue cost
+// per key.  The dense short-context launch (no index list) uses it too once
+// 2 x rows x 64-key chunks reach 8 per SM; below that the 32-key kernel,
+// whose query prologue is a single TMA load, stays ahead.
 //
 // Work unit (one CTA, one per SM): query row r, value half v (latent columns
 // [256v, 256v+256)), split sp (a contiguous range of 64-key chunks of the
@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x < kMaxChunks) misc->vmask[threadIdx.x] = 0ull;
   if (warp == 8) {
     if (lane == 0) {
-      mbar_init(q_full, 1 + 128);  // TMA bytes of blocks 6-8, and the 128 threads writing blocks 0-5
+      // TMA bytes of blocks 6-8, the 128 threads writing blocks 0-5 (+ the test
+      // hook's missing arrival)
+      mbar_init(q_full, 1 + 128 + p.debug_stall);
       for (int s = 0; s < kStages; ++s) {
         mbar_init(kv_full(s), 128);  // one cp.async arrival per gather thread
         mbar_init(kv_empty(s), 1);
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // half a QK sooner (polling between single MMAs measured slower).
     if (lane == 0) {
       int n_qk = 0, n_pv = 0;
-      bool ok = mbar_wait(q_full, 0, abort, kWaitLimitNs);
+      bool ok = mbar_wait(q_full, 0, abort, p.wait_limit_ns);
       // Descriptors differ only in the start-address field (address >> 4 in
       // the low 14 bits, no carry below 256 KiB): built once, offset per MMA.
       const uint64_t qk_a0 = smem_desc(sbase + kOffQ, 16, 1024, kSwizzle128B);
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!progressed && (++spins & 63u) == 0) {  // bounded, like every other wait here
           if (*abort) ok = false;
-          else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          else if (globaltimer_ns() - t0 > p.wait_limit_ns) {
             *abort = 1;
             ok = false;
           }
@@ -364,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = i % kStages;
       const int32_t my_id = next_id;
       if (i + 1 < n_my) next_id = row_id(i + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((i / kStages) & 1) ^ 1, abort, kWaitLimitNs)))
+      if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((i / kStages) & 1) ^ 1, abort, p.wait_limit_ns)))
         break;
 #pragma unroll 2
       for (int rr = 0; rr < 16; ++rr) {
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < n_my; ++i) {
       const int pb = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, abort, kWaitLimitNs));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, abort, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[64];
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, resc)) {
         // O is rescaled in TMEM: every earlier PV must have completed (the
         // last one, PV(i-1), completes after all the others)
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort, kWaitLimitNs));
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort, p.wait_limit_ns));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_wait_st();
       }
       if (i >= 2) {  // P buffer pb was last read by PV(i-2)
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(pb), ((i - 2) >> 1) & 1, abort, kWaitLimitNs));
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(pb), ((i - 2) >> 1) & 1, abort, p.wait_limit_ns));
         if (!ok) break;
       }
       l_run = l_run * alpha + l_chunk;
@@ -476,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(pv_done((n_my - 1) & 1), ((n_my - 1) >> 1) & 1, abort, kWaitLimitNs));
+                      mbar_wait(pv_done((n_my - 1) & 1), ((n_my - 1) >> 1) & 1, abort, p.wait_limit_ns));
     // Every MMA has completed, so the query blocks and key stages are free:
     // the 128 x 256 result is staged there as 128-byte-swizzled boxes of 32
     // fp32 (or 64 bf16) columns, one thread per head row, and written by a
@@ -557,13 +559,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout,
                                    const MlaParams& p, unsigned grid, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(sparse_mla_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  const cudaError_t e = attr.run(
+      [] { return cudaFuncSetAttribute(sparse_mla_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
+  if (e != cudaSuccess) return e;
   return launch_pdl(sparse_mla_wide_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p);
 }
 

@@ -6,11 +6,24 @@
 // position, padded with -1; ties are broken by lower position first and -0.0
 // equals +0.0, so the result is unique and deterministic.
 //
-// One CTA (1024 threads) per query row.  The valid positions of a row are the
-// causal prefix s < L = end_pos - T + t + 1.  Scores are mapped to
-// order-preserving 32-bit keys (larger score = larger key).
+// Kernels, chosen per launch by the score pitch ld (launch_topk):
+//   ld <= 8192 (causal prefill, short decode rows): topk_rows_kernel, one
+//     256-thread CTA per row with the row's keys in registers (16 per thread
+//     up to 4096 positions, 32 above);
+//   8192 < ld <= 131072 (long decode rows): topk_cluster_kernel, one
+//     thread-block cluster per row (8 CTAs of 512 threads for up to three
+//     rows, 4 CTAs of 1024 threads from four rows on), each CTA holding a
+//     slice of the row in shared memory;
+//   ld > 131072: topk_kernel, one 1024-thread CTA per row: the bitmap path
+//     below for rows of up to 131072 valid positions, exact 11/11/10-bit
+//     digit passes over the whole row for longer ones.
+// Scores are mapped to order-preserving 32-bit keys (larger score = larger
+// key); the valid positions of a row are its causal prefix s < L = end_pos -
+// T + t + 1.  Each kernel finds the k-th largest key tau and how many keys
+// equal to tau are kept (the lowest positions), then writes the kept
+// positions ascending.
 //
-// Main path (L <= 131072):
+// topk_kernel's bitmap path:
 //   A. histogram of the top 12 key bits (shared atomics);
 //      a suffix scan finds the bin d* holding the k-th largest key;
 //   B. one pass marks, in a bitmap whose word w covers positions 32w..32w+31
@@ -21,9 +34,9 @@
 //      a scan over a second bitmap);
 //   D. one block scan of the words' popcounts writes the kept positions in
 //      ascending order.
-// Fallback (more candidates than the buffer holds, e.g. massive ties, or
-// very long rows): three 11/11/10-bit digit passes over the whole row and a
-// stable scan-based compaction.
+// Its digit-pass path (rows above 131072 positions, or more candidates than
+// the buffer holds, e.g. massive ties): three 11/11/10-bit digit passes over
+// the whole row and a stable scan-based compaction.
 #include <cooperative_groups.h>
 
 #include "dsa_internal.h"
@@ -881,14 +894,13 @@ template <int CS>
 int launch_cluster(const TopkArgs& a, cudaStream_t stream) {
   auto kern = topk_cluster_kernel<CS>;
   const size_t smem = sizeof(ClusterSmem<CS>);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    if (CS > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  static PerDeviceOnce attrs_set;  // per template instance
+  if (attrs_set.run([&] {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess && CS > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        return e;
+      }) != cudaSuccess)
+    return DSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.B * a.T * CS));
   cfg.blockDim = dim3(ClusterCfg<CS>::kThreads);
@@ -931,13 +943,10 @@ int launch_topk(const TopkArgs& a, cudaStream_t stream) {
                                      a.scores, a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
     return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  if (attr.run([] { return cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes); }) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   const cudaError_t e = launch_pdl(topk_kernel, dim3(rows), dim3(kThreads), kSmemBytes, stream, a.scores,
                                    a.ld, a.offsets, a.B, a.T, a.k, a.indices, a.status);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

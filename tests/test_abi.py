@@ -109,3 +109,12 @@ def test_workspace_sizes(L):
     args = [P(A), P(A), P(A), None, 0, P(A), P(A), P(A), 1, 32768, 32768, 2048, 128, 0.07, P(A), 0,
             None, P(A), 1024, None, None]
     assert f(*args) == 3
+
+
+def test_stall_hook_rejects_bad_limits(L):
+    """The timeout test hook checks its arguments on the host."""
+    f = L.lib.dsa_debug_stall_attention
+    assert f(1, 10) == 1                # limit below 1 ms
+    assert f(1, 5 * 10 ** 9) == 1       # above 1 s
+    assert f(-1, 5_000_000) == 1        # negative count
+    assert f(0, 0) == 0                 # cancel

@@ -271,6 +271,66 @@ def test_sparse_mla_closed_forms():
     assert torch.all(out3 == 0) and torch.all(torch.isinf(lse3))
 
 
+def _ragged_mla_case(eps, T, H, seed):
+    """B = len(eps) sequences packed one after another in one cache, preceded
+    by 3 rows no sequence owns (so a dropped base offset reads other rows)."""
+    B = len(eps)
+    q = _bf16((B, T, H, 576), seed + 1)
+    pad = 3
+    kv = _bf16((pad + sum(eps), 576), seed + 2)
+    off = _offsets(eps) + pad
+    return q, kv, off
+
+
+def test_ragged_mla_sequences_use_their_own_cache_slice():
+    """[Mask] decode listing: each sequence attends over its own kv_cache[:end_pos].
+    With B = 3 ragged sequences in one cache, every row of sequence b must equal
+    (1) the same oracle call on sequence b alone, with its slice of the cache as
+    the whole cache, and (2) torch SDPA over that slice (sparse: the rows the
+    index list names; dense: the causal prefix).  A missing or doubled base
+    offset off[b] reads another sequence's rows and fails both."""
+    eps, T, H, k, scale = [17, 40, 9], 2, 3, 12, 0.11
+    B = len(eps)
+    q, kv, off = _ragged_mla_case(eps, T, H, seed=21)
+    g = torch.Generator().manual_seed(22)
+    idx = torch.full((B * T, k), -1, dtype=torch.int32)
+    for b, E in enumerate(eps):
+        for t in range(T):
+            n = min(k, E - 1)
+            sel = torch.randperm(E, generator=g)[:n].to(torch.int32)
+            idx[b * T + t, :n] = sel                      # unsorted, -1 holes at the end
+    sp, lsp = oracle.sparse_mla(q, kv, off, idx, B, T, H, k, scale)
+    de, lde = oracle.dense_mla(q, kv, off, B, T, H, scale)
+    for b, E in enumerate(eps):
+        lo = int(off[b])
+        sl = kv[lo:lo + E].contiguous()
+        one = _offsets([E])
+        rows = slice(b * T, (b + 1) * T)
+        sp1, lsp1 = oracle.sparse_mla(q[b:b + 1].contiguous(), sl, one, idx[rows].contiguous(), 1, T, H, k, scale)
+        de1, lde1 = oracle.dense_mla(q[b:b + 1].contiguous(), sl, one, 1, T, H, scale)
+        torch.testing.assert_close(sp[rows], sp1, rtol=0, atol=0)
+        torch.testing.assert_close(lsp[rows], lsp1, rtol=0, atol=0)
+        torch.testing.assert_close(de[rows], de1, rtol=0, atol=0)
+        torch.testing.assert_close(lde[rows], lde1, rtol=0, atol=0)
+        # torch SDPA over the slice: K = row[:576], V = row[:512]
+        Q = q[b].double().permute(1, 0, 2)                # [H,T,576]
+        K = sl.double()[None].expand(H, E, 576)
+        V = sl.double()[:, :512][None].expand(H, E, 512)
+        causal = torch.tensor([[s <= E - T + t for s in range(E)] for t in range(T)])
+        ref_d = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=causal, scale=scale)
+        torch.testing.assert_close(de[rows], ref_d.permute(1, 0, 2), rtol=1e-10, atol=1e-12)
+        chosen = torch.zeros(T, E, dtype=torch.bool)
+        for t in range(T):
+            for s in idx[b * T + t].tolist():
+                if s >= 0:
+                    chosen[t, s] = True
+        ref_s = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=chosen, scale=scale)
+        torch.testing.assert_close(sp[rows], ref_s.permute(1, 0, 2), rtol=1e-10, atol=1e-12)
+        logits = (Q @ K.transpose(-1, -2)) * scale
+        ref_lse = torch.logsumexp(logits.masked_fill(~chosen, -math.inf), dim=-1).permute(1, 0)
+        torch.testing.assert_close(lsp[rows], ref_lse, rtol=1e-12, atol=1e-12)
+
+
 def test_sparse_mla_rejects_out_of_range_indices():
     q, kv, off = _mla_case(10, 1, 2)
     with pytest.raises(ValueError):
