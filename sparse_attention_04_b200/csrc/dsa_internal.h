@@ -138,6 +138,13 @@ constexpr int kMlaWideChunk = 64;
 cudaError_t launch_sparse_mla_wide(const CUtensorMap& tq, const CUtensorMap& tout,
                                    const MlaParams& p, unsigned grid, cudaStream_t stream);
 
+// The attention kernel for launches with many 128-key chunks per SM
+// (sparse_mla_pair.cu): a cluster of two CTAs per (row, split), the QK side
+// and the PV side; grid of 2 CTAs per unit.
+constexpr int kMlaPairChunk = 128;
+cudaError_t launch_sparse_mla_pair(const CUtensorMap& tq, const CUtensorMap& tout, const MlaParams& p,
+                                   unsigned n_units, cudaStream_t stream);
+
 int mla_num_splits(int n_rows, int k, int H, bool dense);  // dense: no index list (short context)
 int mla_chunk(int n_rows, int k, bool dense);
 size_t mla_workspace_bytes(int n_rows, int H, int k);

@@ -32,6 +32,8 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
+#include <cstring>
 
 #include "dsa_internal.h"
 #include "sm100.cuh"
@@ -576,49 +578,81 @@ __global__ void __launch_bounds__(64)
 
 }  // namespace
 
-// Which attention kernel a launch uses.  The 64-key kernel halves the QK
-// issue cost per key, and after a selection stage it is the faster one for
-// any row count (decode 32K: 27.9 against 29.5 us per step; four 131K rows:
-// 49.0 against 52.1 us).  Its query prologue (blocks 0-5 into TMEM through
+// Which attention kernel a launch uses.
+//
+// The pair kernel (sparse_mla_pair.cu: a QK CTA and a PV CTA per (row,
+// split), 128-key chunks, S computed once at N = 128) wherever the launch has
+// at least kMlaPairMinChunksPerSlot 128-key chunks per cluster slot (two SMs):
+// large decode batches and causal prefill.  Its per-unit prologue (128 KB of
+// query into TMEM) and its 128-key chunks make it slower for a few long rows.
+//
+// Otherwise the 64-key kernel, which halves the QK issue cost per key of the
+// 32-key kernel and after a selection stage is the faster one for any row
+// count (decode 32K: 27.9 against 29.5 us per step; four 131K rows: 49.0
+// against 52.1 us).  Its query prologue (blocks 0-5 into TMEM through
 // registers) is slower than the 32-key kernel's single TMA load, and only a
 // launch with no preceding stage to hide behind pays for it: the dense
 // short-context attention with few chunks per SM (one 2K row: 14.6 against
 // 13.9 us) keeps the 32-key kernel unless 2 * rows * 64-key chunks reaches
 // kMlaWideMinChunksPerSm times the SM count.
+//
+// DSA_ATTENTION_KERNEL=pair|wide|narrow in the environment (read once per
+// process) forces one of the three for every launch, for measurements.
 constexpr int kMlaWideMinChunksPerSm = 8;
+constexpr int kMlaPairMinChunksPerSlot = 4;
+
+namespace {
+int forced_kernel() {  // 0: automatic, else the forced chunk size
+  static const int forced = [] {
+    const char* e = std::getenv("DSA_ATTENTION_KERNEL");
+    if (!e) return 0;
+    if (!std::strcmp(e, "pair")) return kMlaPairChunk;
+    if (!std::strcmp(e, "wide")) return kMlaWideChunk;
+    if (!std::strcmp(e, "narrow")) return kChunk;
+    return 0;
+  }();
+  return forced;
+}
+}  // namespace
 
 int mla_chunk(int n_rows, int k, bool dense) {
+  if (const int f = forced_kernel()) return f;
+  const int64_t sms = device_info().sm_count;
+  const int64_t n128 = (k + kMlaPairChunk - 1) / kMlaPairChunk;
+  if ((int64_t)n_rows * n128 >= kMlaPairMinChunksPerSlot * (sms / 2)) return kMlaPairChunk;
   if (!dense) return kMlaWideChunk;
   const int64_t n64 = (k + kMlaWideChunk - 1) / kMlaWideChunk;
-  const int64_t sms = device_info().sm_count;
   return 2 * (int64_t)n_rows * n64 >= kMlaWideMinChunksPerSm * sms ? kMlaWideChunk : kChunk;
 }
 
 // Splits of a row's index list.  Every split is a pair of CTAs (one per value
-// half, one CTA per SM for shared memory), so n_rows x splits x 2 CTAs run in
-// ceil(that / SMs) waves, each costing its chunks (1000 per 32 keys) plus
-// about 1500 of fixed work (query tile, epilogue); every (row, split) partial
-// costs the combine about 17 at H = 128 (measured on B200).  The split count
-// minimises that estimate, ties going to fewer splits, with at least 64 keys
-// per split (fewer keys per split double the partials' traffic for too
-// little gain).
+// half, or the QK and PV sides of the pair kernel; one CTA per SM for shared
+// memory), so n_rows x splits x 2 CTAs run in ceil(that / SMs) waves, each
+// costing its chunks (1000 per 32 keys for the 32- and 64-key kernels, 1000
+// per 64 keys for the pair kernel) plus about 1500 of fixed work (query tile,
+// epilogue; 2500 for the pair kernel); every (row, split) partial costs the
+// combine about 17 at H = 128 (measured on B200).  The split count minimises
+// that estimate, ties going to fewer splits, with at least 64 keys per split
+// (fewer keys per split double the partials' traffic for too little gain).
 static_assert(DSA_MAX_TOPK / 64 <= kMaxSplits, "the combine holds every split of a row in registers");
 
 int mla_num_splits(int n_rows, int k, int H, bool dense) {
   const int chunk = mla_chunk(n_rows, k, dense);
+  const bool pair = chunk == kMlaPairChunk;
   const int n_chunks = (k + chunk - 1) / chunk;
   const int64_t sms = device_info().sm_count;
   int max_splits = n_chunks * chunk / 64;
   if (max_splits > n_chunks) max_splits = n_chunks;
   if (max_splits < 1) max_splits = 1;
+  const int64_t per_chunk = pair ? 2000 : 1000 * (int64_t)chunk / 32;
+  const int64_t fixed = pair ? 2500 : 1500;
   int best = 1;
   int64_t best_cost = -1;
   for (int ns = 1; ns <= max_splits; ++ns) {
     const int cps = (n_chunks + ns - 1) / ns;
     if ((n_chunks + cps - 1) / cps != ns) continue;  // same chunks per split as a smaller count
     const int64_t waves = ((int64_t)n_rows * ns * 2 + sms - 1) / sms;
-    const int64_t cost = waves * (1000 * (int64_t)cps * chunk / 32 + 1500) +
-                         (ns > 1 ? (int64_t)n_rows * ns * 17 * H / 128 : 0);
+    const int64_t cost = waves * (per_chunk * cps + fixed) + (ns > 1 ? (int64_t)n_rows * ns * 17 * H / 128 : 0);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = ns;
@@ -712,9 +746,10 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
     return DSA_ERR_CUDA;
   const int64_t grid = (int64_t)n_rows * ns * 2;
   const cudaError_t e =
-      chunk == kMlaWideChunk
-          ? launch_sparse_mla_wide(tq, tout, p, (unsigned)grid, stream)
-          : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, tout, p);
+      chunk == kMlaPairChunk   ? launch_sparse_mla_pair(tq, tout, p, (unsigned)(grid / 2), stream)
+      : chunk == kMlaWideChunk ? launch_sparse_mla_wide(tq, tout, p, (unsigned)grid, stream)
+                               : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes,
+                                            stream, tq, tout, p);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (ns > 1) {
     if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(64), 0, stream,
