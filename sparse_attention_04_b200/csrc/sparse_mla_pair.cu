@@ -465,8 +465,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // staged as P row h (K-major without swizzle: 8-row x 16-byte core
       // matrices, 128 bytes apart along K, 2048 apart along M); returns the
       // sum of the rounded values.
+      // (Four partial sums: one serial chain of 32 additions would bound
+      // the loop by its latency.)
       auto emit = [&](const uint32_t (&sv)[64], uint8_t* prow, int half, float m_sub) -> float {
-        float2 l2 = make_float2(0.f, 0.f);
+        float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 nm2 = make_float2(-m_sub, -m_sub);
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
@@ -476,12 +478,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int j = 8 * c8 + 2 * e;
             const float2 d = __fadd2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), nm2);
             const __nv_bfloat162 pb = __floats2bfloat162_rn(ex2_approx(d.x), ex2_approx(d.y));
-            l2 = __fadd2_rn(l2, __bfloat1622float2(pb));
+            l2[e] = __fadd2_rn(l2[e], __bfloat1622float2(pb));
             w4[e] = *reinterpret_cast<const uint32_t*>(&pb);
           }
           *reinterpret_cast<uint4*>(prow + (8 * half + c8) * 128) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        return l2.x + l2.y;
+        const float2 a = __fadd2_rn(l2[0], l2[1]), b = __fadd2_rn(l2[2], l2[3]);
+        return (a.x + b.x) + (a.y + b.y);
+      };
+      // max of 64 values as a tree (a serial chain of 64 would bound the loop)
+      auto max64 = [](const uint32_t (&sv)[64]) -> float {
+        float m8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          m8[q] = __uint_as_float(sv[q]);
+#pragma unroll
+          for (int j = 8 + q; j < 64; j += 8) m8[q] = fmaxf(m8[q], __uint_as_float(sv[j]));
+        }
+        return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       };
       for (int i = 0; i < n_my; ++i) {
         const int sb = i & 1;  // S buffer, staging buffer and CTA 1's message buffer
@@ -508,8 +522,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld64(s_addr + 64 * half, sv);
           tc_wait_ld();
           scaled(sv, i, half);
-#pragma unroll
-          for (int j = 0; j < 64; ++j) mc = fmaxf(mc, __uint_as_float(sv[j]));
+          mc = fmaxf(mc, max64(sv));
           l_chunk += emit(sv, prow, half, m_sub0);
         }
         float alpha = 1.f;
