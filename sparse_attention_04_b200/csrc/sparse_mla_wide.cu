@@ -53,8 +53,8 @@ constexpr int kOffQ = 0;
 constexpr int kOffKv = kOffQ + kQBytes;
 constexpr int kOffP = kOffKv + kStages * kKvBytes;  // two P buffers
 constexpr int kOffBar = kOffP + 2 * kPBytes;
-// q_full, kv_full[2], kv_empty[2], s_full, s_empty, p_full[2], pv_done[2], drain
-constexpr int kNumBar = 12;
+// q_full, kv_full[2], kv_empty[2], s_full, s_empty, p_full[2], pv_done[2], drain, kv_first
+constexpr int kNumBar = 13;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
 constexpr int kStageBlock = 128 * 128;              // epilogue staging: one box, 128 rows x 128 B
 static_assert(8 * kStageBlock <= kOffP, "the staged output fits where the query blocks and key stages were");
@@ -101,6 +101,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_full = [&](int b) { return bar0 + 8u * (7 + b); };
   auto pv_done = [&](int b) { return bar0 + 8u * (9 + b); };
   const uint32_t drain = bar0 + 8u * 11;
+  // The split's first chunk is gathered into stage 0 by warps 0-7 together
+  // (the softmax warps are idle until its scores exist), with its own
+  // barrier; stage 0's kv_full phases then start at chunk 2.
+  const uint32_t kv_first = bar0 + 8u * 12;
   MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
   volatile int* abort = &misc->abort;
 
@@ -146,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(pv_done(i), 1);
       }
       mbar_init(drain, 1);
+      mbar_init(kv_first, 256);
       fence_mbar_init();
       if (geo_ok) {
         mbar_arrive_expect_tx(q_full, kQBytes);
@@ -192,6 +197,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   grid_dependency_wait();  // the indices come from the previous kernel
   allow_dependents_launch();
+
+  // ---- the split's first chunk: warps 0-7 copy 8 rows each into stage 0
+  // right away, before the validity pass below (a single SM's gather rate
+  // grows with the threads issuing it; a decode row's split often has just
+  // this one chunk).  Invalid positions are zero-filled.
+  if (geo_ok && warp < 8) {
+    const int pos0 = c_begin * kChunk + 8 * warp + lane;
+    const int32_t my_id = (lane < 8 && pos0 < p.k) ? selected_pos(idx_row, dense, pos0, L_row) : -1;
+#pragma unroll 2
+    for (int rr = 0; rr < 8; ++rr) {
+      const int jr = 8 * warp + rr;
+      const int32_t id = __shfl_sync(0xffffffffu, my_id, rr);
+      const bool valid = index_ok(id, E);
+      const __nv_bfloat16* src = valid ? p.kv + ((int64_t)base_row + id) * kDQK : p.kv;
+      const uint32_t dst_row = sbase + kOffKv + (jr >> 3) * 1024 + (jr & 7) * 128;
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int c = lane + 32 * u;  // 16-byte piece of the 72 in a row
+        if (c < kDQK / 8) {
+          const int kb = c >> 3, cc = c & 7;
+          cp_async_16(dst_row + kb * kBlockBytes + ((cc ^ (jr & 7)) << 4), src + c * 8, valid ? 16u : 0u);
+        }
+      }
+    }
+    cp_async_mbar_arrive(kv_first);
+  }
 
   // ---- how many chunks of this split hold a selected row.  Each warp owns
   // whole chunks: it loads all their indices first (one L2 round trip), then
@@ -253,9 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (warp == 8 && lane == 0 && geo_ok) {  // the query tile must land before the CTA exits
+    if (warp == 8 && lane == 0 && geo_ok) {  // the query tile and the first chunk must land before the CTA exits
       volatile int never = 0;
       mbar_wait(q_full, 0, &never, 10000000ull);
+      mbar_wait(kv_first, 0, &never, 10000000ull);
     }
   } else if (warp == 8) {
     // -------------------------------------------------------------- MMA issuer
@@ -277,6 +309,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qk_b0 = smem_desc(sbase + kOffKv, 16, 1024, kSwizzle128B);
       const uint64_t pv_a0 = smem_desc(sbase + kOffP, 128, 1024, kSwizzleNone);
       const uint64_t pv_b0 = smem_desc(sbase + kOffKv + (4 * v) * kBlockBytes, kBlockBytes, 1024, kSwizzle128B);
+      // chunk i has landed: the first chunk on its own barrier, stage 0's
+      // later chunks (2, 4, ...) on kv_full(0) phases 0, 1, ...
+      auto kv_ready = [&](int i) -> bool {
+        if (i == 0) return mbar_try_wait(kv_first, 0);
+        const int st = i % kStages;
+        return mbar_try_wait(kv_full(st), (i / kStages - (st == 0 ? 1 : 0)) & 1);
+      };
       // PV of chunk n_pv (its P is in shared memory; p_full has been seen)
       auto issue_pv = [&]() {
         const int j = n_pv;
@@ -295,8 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t spins = 0;
       while (ok && n_pv < n_my) {
         bool progressed = false;
-        if (n_qk < n_my && (n_qk == 0 || mbar_try_wait(s_empty, (n_qk - 1) & 1)) &&
-            mbar_try_wait(kv_full(n_qk % kStages), (n_qk / kStages) & 1)) {
+        if (n_qk < n_my && (n_qk == 0 || mbar_try_wait(s_empty, (n_qk - 1) & 1)) && kv_ready(n_qk)) {
           const int st = n_qk % kStages;
           fence_proxy_async_smem();  // rows written by cp.async, read by the tensor core
           tc_fence_after();
@@ -345,15 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(drain);
         mbar_wait(drain, 0, &never, 10000000ull);
         mbar_wait(q_full, 0, &never, 10000000ull);
+        mbar_wait(kv_first, 0, &never, 10000000ull);
       }
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- row gather
-    // Warp 4 + gw copies rows 16gw .. 16gw+15 of every chunk, one row at a
-    // time, so each copy instruction reads 512 contiguous bytes of a row.
-    // Completion is signalled by the copies themselves (cp.async arrival
-    // on the stage's barrier), so both stages are in flight from the start;
-    // the next chunk's indices are read while the current one is issued.
+    // From the second chunk on (the first was copied above), warp 4 + gw
+    // copies rows 16gw .. 16gw+15 of every chunk, one row at a time, so each
+    // copy instruction reads 512 contiguous bytes of a row.  Completion is
+    // signalled by the copies themselves (cp.async arrival on the stage's
+    // barrier), so both stages are in flight from the start; the next
+    // chunk's indices are read while the current one is issued.
     const int gw = warp - 4;
     const __nv_bfloat16* kv = p.kv;
     auto row_id = [&](int i) -> int32_t {
@@ -361,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos = (c_begin + i) * kChunk + gw * 16 + lane;
       return pos < p.k ? selected_pos(idx_row, dense, pos, L_row) : -1;
     };
-    int32_t next_id = row_id(0);
-    for (int i = 0; i < n_my; ++i) {
+    int32_t next_id = n_my > 1 ? row_id(1) : -1;
+    for (int i = 1; i < n_my; ++i) {
       const int st = i % kStages;
       const int32_t my_id = next_id;
       if (i + 1 < n_my) next_id = row_id(i + 1);
@@ -546,6 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) bulk_wait_read();  // the staged boxes stay valid until read
   }
 
+  cp_async_wait<0>();  // the first chunk's copies of warps 0-7
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
