@@ -487,8 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
-// One CTA of 64 threads per (row, head); thread c owns eight columns and
-// issues the 16-byte loads of 32 splits at once.
+// G heads of one row per CTA, 64 threads per head; thread c of a head owns
+// eight columns and issues the 16-byte loads of 32 splits at once (16 when
+// G > 1, for registers).  G > 1
+// serves launches with many (row, head) pairs: one CTA per pair would be so
+// short that the rate at which CTAs are dispatched sets the time (32 rows x
+// 128 heads, two splits: 19 us with one head per CTA, measured on B200).
 constexpr int kMaxSplits = 64;
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -500,24 +504,31 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float
   }
 }
 
-__global__ void __launch_bounds__(64)
+template <int G>
+__global__ void __launch_bounds__(64 * G)
     mla_combine_kernel(const __nv_bfloat16* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
-  __shared__ float s_w[kMaxSplits];
-  __shared__ float s_ml[2];
+  __shared__ float s_w[G][kMaxSplits];
+  __shared__ float s_ml[G][2];
   grid_dependency_wait();  // partials come from the previous kernel
   allow_dependents_launch();
-  const int64_t rh = blockIdx.x;  // row * H + head
-  const int64_t r = rh / H, h = rh % H;
-  const int c8 = threadIdx.x;  // eight columns: 8*c8 .. 8*c8+7
-  const uint4* base = reinterpret_cast<const uint4*>(ws_o + (r * n_splits * H + h) * kDV) + c8;
+  const int groups = (H + G - 1) / G;  // head groups per row
+  const int64_t r = blockIdx.x / groups;
+  const int g = threadIdx.x >> 6;      // head of the group
+  const int64_t h = (int64_t)(blockIdx.x % groups) * G + g;
+  const bool live = h < H;             // uniform over the head's two warps
+  const int64_t rh = r * H + h;
+  const int c8 = threadIdx.x & 63;  // eight columns: 8*c8 .. 8*c8+7
+  const uint4* base = reinterpret_cast<const uint4*>(ws_o + (r * n_splits * H + (live ? h : 0)) * kDV) + c8;
   const int64_t stride = (int64_t)H * kDV / 8;  // uint4 between consecutive splits
-  uint4 o[32];
+  // splits whose loads are in flight at once (registers: 512 threads at G = 8)
+  constexpr int NB = G == 1 ? 32 : 16;
+  uint4 o[NB];
 #pragma unroll
-  for (int s = 0; s < 32; ++s)
-    if (s < n_splits) o[s] = __ldg(base + s * stride);
-  if (threadIdx.x < 32) {
-    const int s0 = threadIdx.x, s1 = threadIdx.x + 32;
+  for (int s = 0; s < NB; ++s)
+    if (live && s < n_splits) o[s] = __ldg(base + s * stride);
+  if (live && c8 < 32) {
+    const int s0 = c8, s1 = c8 + 32;
     float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
     if (s0 < n_splits) {
       const int64_t slot = (r * n_splits + s0) * H + h;
@@ -537,26 +548,26 @@ __global__ void __launch_bounds__(64)
     float L = l0 * f0 + l1 * f1;
 #pragma unroll
     for (int d = 16; d; d >>= 1) L += __shfl_xor_sync(0xffffffffu, L, d);
-    s_w[s0] = f0;
-    s_w[s1] = f1;
+    s_w[g][s0] = f0;
+    s_w[g][s1] = f1;
     if (s0 == 0) {
-      s_ml[0] = M;
-      s_ml[1] = L;
+      s_ml[g][0] = M;
+      s_ml[g][1] = L;
     }
   }
   __syncthreads();
-  const float M = s_ml[0], L = s_ml[1];
+  if (!live) return;  // no barrier below
+  const float M = s_ml[g][0], L = s_ml[g][1];
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int sb = 0; sb < n_splits; sb += NB) {
+    if (sb > 0) {  // the next group of splits
 #pragma unroll
-  for (int s = 0; s < 32; ++s)
-    if (s < n_splits) acc_bf16x8(acc, o[s], s_w[s]);
-  if (n_splits > 32) {  // the second group of splits
+      for (int s = 0; s < NB; ++s)
+        if (sb + s < n_splits) o[s] = __ldg(base + (sb + s) * stride);
+    }
 #pragma unroll
-    for (int s = 0; s < 32; ++s)
-      if (32 + s < n_splits) o[s] = __ldg(base + (32 + s) * stride);
-#pragma unroll
-    for (int s = 0; s < 32; ++s)
-      if (32 + s < n_splits) acc_bf16x8(acc, o[s], s_w[32 + s]);
+    for (int s = 0; s < NB; ++s)
+      if (sb + s < n_splits) acc_bf16x8(acc, o[s], s_w[g][sb + s]);
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if (out_bf16) {
@@ -573,7 +584,28 @@ __global__ void __launch_bounds__(64)
     o4[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     o4[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
   }
-  if (threadIdx.x == 0 && lse) lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  if (c8 == 0 && lse) lse[rh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+// Heads per combine CTA: one while that leaves at least two CTAs per SM,
+// else up to eight.
+int combine_heads_per_cta(int64_t n_rows, int H, int sms) {
+  int G = 1;
+  while (G < 8 && n_rows * ((H + 2 * G - 1) / (2 * G)) >= 2 * (int64_t)sms) G *= 2;
+  return G;
+}
+
+cudaError_t launch_combine(const MlaParams& p, int64_t n_rows, int H, cudaStream_t stream) {
+  const int G = combine_heads_per_cta(n_rows, H, device_info().sm_count);
+  const dim3 grid((unsigned)(n_rows * ((H + G - 1) / G)));
+  const __nv_bfloat16* o = p.ws_o;
+  const float* ml = p.ws_ml;
+  switch (G) {
+    case 1: return launch_pdl(mla_combine_kernel<1>, grid, dim3(64), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
+    case 2: return launch_pdl(mla_combine_kernel<2>, grid, dim3(128), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
+    case 4: return launch_pdl(mla_combine_kernel<4>, grid, dim3(256), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
+    default: return launch_pdl(mla_combine_kernel<8>, grid, dim3(512), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
+  }
 }
 
 }  // namespace
@@ -751,12 +783,7 @@ int launch_sparse_mla(const MlaArgs& a, cudaStream_t stream) {
                                : launch_pdl(sparse_mla_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes,
                                             stream, tq, tout, p);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
-  if (ns > 1) {
-    if (launch_pdl(mla_combine_kernel, dim3((unsigned)((int64_t)n_rows * a.H)), dim3(64), 0, stream,
-                   (const __nv_bfloat16*)p.ws_o, (const float*)p.ws_ml, a.H, ns, a.out, p.out_bf16, a.lse) !=
-        cudaSuccess)
-      return DSA_ERR_CUDA;
-  }
+  if (ns > 1 && launch_combine(p, n_rows, a.H, stream) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }
 

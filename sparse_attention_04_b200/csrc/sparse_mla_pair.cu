@@ -16,15 +16,15 @@
 //
 //   CTA 0 (QK side).  Query blocks 0-7 (latent 0-511) sit in TMEM as the A
 //     operand of S, block 8 (rope) in shared memory.  The chunk's rows stream
-//     through a ring of four 48 KB slots, each three 64-column blocks of the
+//     through a ring of three 48 KB slots, each three 64-column blocks of the
 //     128 rows (swizzled, K-major); every slot is read once by the QK MMAs.
 //     S goes to one of two 128-column TMEM buffers.  Softmax runs in
 //     registers, thread = head = TMEM lane, with the lazy running max of
 //     sparse_mla.cu (raised only when a chunk exceeds it by more than 2^8).
-//     Each thread stores its bf16 P row and its rescale factor into CTA 1's
-//     shared memory with asynchronous distributed-shared-memory stores
-//     (st.async), whose bytes complete on CTA 1's barrier; the thread moves on
-//     to the next chunk without waiting for them.
+//     Each thread writes its bf16 P row and its rescale factor into one of
+//     two local staging buffers and moves on to the next chunk; warp 15 sends
+//     each staged message to CTA 1 with one bulk copy (shared::cta to
+//     shared::cluster), whose bytes complete on CTA 1's barrier.
 //   CTA 1 (PV side).  O (128 heads x 512 latent, fp32) fills all 512 TMEM
 //     columns.  The chunk's latent columns 0-511 stream through a ring of
 //     four 32 KB slots (two 64-column blocks each).  Before P.V of a chunk
@@ -40,7 +40,8 @@
 // once per key instead of twice, at N = 128 instead of 64.
 //
 // Roles in each CTA: warps 0-3 softmax (CTA 0) or rescale + epilogue (CTA 1),
-// warp 12 TMEM allocator + MMA issuer, warps 4-11 and 13-15 row gather.
+// warp 12 TMEM allocator + MMA issuer, warp 15 message sender (CTA 0), the
+// other warps (4-11, 13-14; and 15 in CTA 1) row gather.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -106,7 +107,7 @@ constexpr int kSmemBytes = kOffMisc + (int)sizeof(PairMisc) + 1024;
 // cp.async gather rate grows with the number of threads issuing it (about 35,
 // 55 and 75 GB/s with 128, 256 and 384 threads, measured on B200), so most of
 // the CTA gathers.  512 threads leave 128 registers per thread; the softmax
-// therefore holds 32 scores at a time.
+// therefore holds one 64-column half of a row's scores at a time.
 constexpr int kThreads = 512;
 constexpr int kMmaWarp = 12;
 constexpr int kSendWarp = 15;  // CTA 0 only; a gather warp in CTA 1

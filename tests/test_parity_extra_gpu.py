@@ -3,6 +3,8 @@ device-side timeout path.
 
   - the e4m3 indexer with T > 1 (causal prefill rows of ragged sequences);
   - the attention at head counts other than 16 and 128, both output types;
+  - the combine with several heads per CTA (a partly filled last group);
+  - split rows on a workspace that starts zero, all ones or random, reused;
   - a short-context decode step whose query was written by the kernel copy
     just before it on the same stream;
   - a pipeline wait that runs out (test hook), then a normal call.
@@ -76,6 +78,37 @@ def test_attention_head_counts(cuda_device, H, out_dtype):
     check_mla(out.reshape(B, H, -1), lse.reshape(B, H), idx, sub, list(range(B)))
 
 
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_combine_several_heads_per_cta(cuda_device, out_dtype):
+    """32 rows at H = 100, k = 2048: two splits per row and a combine with
+    eight heads per CTA, whose last group of each row holds four heads past
+    H (they must write nothing).  Rows checked against the oracle; every
+    output row must be finite."""
+    L = _lib()
+    B, H, k = 32, 100, 2048
+    wl = dsa_inputs.custom("comb_g", B=B, end_pos=None, end_pos_range=(2100, 6000), topk=k, H=H,
+                           out_dtype=out_dtype, scale=192 ** -0.5, seed=91)
+    inp = dsa_inputs.make_inputs(wl, cuda_device)
+    g = torch.Generator().manual_seed(92)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k].sort().values.to(torch.int32) for E in inp.end_pos])
+    idx = idx.to(cuda_device)
+    dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    out = torch.full((B + 1, 1, H, 512), float("nan"), dtype=dt, device=cuda_device)  # + a guard row
+    lse = torch.full((B + 1, 1, H), float("nan"), dtype=torch.float32, device=cuda_device)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ws = torch.empty(max(16, L.sparse_mla_workspace_size(B, 1, H, k)), dtype=torch.uint8, device=cuda_device)
+    L.sparse_mla(inp.q, inp.kv, inp.offsets, idx, B, 1, H, k, wl.scale, inp.rows, out[:B], lse=lse[:B],
+                 workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, _lib_status(st)
+    assert torch.isfinite(out[:B].float()).all() and torch.isfinite(lse[:B]).all()
+    assert torch.isnan(out[B].float()).all() and torch.isnan(lse[B]).all()  # nothing written past the rows
+    rows = [0, 13, 31]
+    sub = subset(inp, rows)
+    check_mla(out[rows].reshape(len(rows), H, -1), lse[rows].reshape(len(rows), H), idx[rows], sub,
+              list(range(len(rows))))
+
+
 @pytest.mark.parametrize("H", [1, 5, 64, 100])
 def test_short_context_head_counts(cuda_device, H):
     """The decode step's dense short-context attention at the same head counts."""
@@ -91,6 +124,43 @@ def test_short_context_head_counts(cuda_device, H):
     for b, E in enumerate(sub.end_pos):
         full[b, :E] = torch.arange(E, dtype=torch.int32)
     check_mla(res.out.reshape(2, H, -1), res.lse.reshape(2, H), full, sub, [0, 1])
+
+
+# ------------------------------------------------------------------ split rows on a reused workspace
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, None])
+def test_split_rows_on_reused_workspace(cuda_device, fill):
+    """Two 20K rows, k = 2048: the 64-key kernel splits each row 32 ways and
+    the combine merges the partials.  The workspace starts all zero, all ones
+    or random; three calls with different index lists then run on it back to
+    back (the last with empty later splits), and each must match the oracle:
+    nothing a call reads may come from what an earlier call left there."""
+    L = _lib()
+    B, H, k = 2, 128, 2048
+    wl = dsa_inputs.custom("reuse_ws", B=B, end_pos=20000, topk=k, H=H, out_dtype="bf16",
+                           scale=192 ** -0.5, seed=101)
+    inp = dsa_inputs.make_inputs(wl, cuda_device)
+    nbytes = L.sparse_mla_workspace_size(B, 1, H, k)
+    assert nbytes > 0
+    if fill is None:
+        ws = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, generator=torch.Generator().manual_seed(3))
+        ws = ws.to(cuda_device)
+    else:
+        ws = torch.full((nbytes,), fill, dtype=torch.uint8, device=cuda_device)
+    sub = subset(inp, [0, 1])
+    g = torch.Generator().manual_seed(102)
+    for call in range(3):
+        idx = torch.stack([torch.randperm(E, generator=g)[:k].sort().values.to(torch.int32) for E in inp.end_pos])
+        if call == 2:
+            idx[1, 1000:] = -1  # later splits of row 1 hold nothing
+        out = torch.full((B, 1, H, 512), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+        lse = torch.empty(B, 1, H, dtype=torch.float32, device=cuda_device)
+        st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        L.sparse_mla(inp.q, inp.kv, inp.offsets, idx.to(cuda_device), B, 1, H, k, wl.scale, inp.rows, out,
+                     lse=lse, workspace=ws, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0, _lib_status(st)
+        check_mla(out.reshape(B, H, -1), lse.reshape(B, H), idx, sub, [0, 1])
 
 
 # ------------------------------------------------------------------ ordering after a copy kernel
