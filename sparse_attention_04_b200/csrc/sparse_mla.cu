@@ -487,12 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merges the per-split partials of one (row, head): O = sum_s 2^(m_s-M) O_s /
 // sum_s 2^(m_s-M) l_s (the same log-sum-exp merge a single pass would do).
-// G heads of one row per CTA, 64 threads per head; thread c of a head owns
-// eight columns and issues the 16-byte loads of 32 splits at once (16 when
-// G > 1, for registers).  G > 1
-// serves launches with many (row, head) pairs: one CTA per pair would be so
-// short that the rate at which CTAs are dispatched sets the time (32 rows x
-// 128 heads, two splits: 19 us with one head per CTA, measured on B200).
+// G heads of one row per CTA, 64 * SP threads per head: thread (part, c)
+// owns eight columns c and the splits part, part + SP, ...; with SP > 1 the
+// parts' sums meet in shared memory.  Launch shapes:
+//   - many (row, head) pairs: G > 1, SP = 1.  One CTA per pair would be so
+//     short that the rate at which CTAs are dispatched sets the time (32 rows
+//     x 128 heads, two splits: 19 us with one head per CTA, measured on B200);
+//   - few pairs with many splits (a decode row): G = 1, SP = 4, so that four
+//     times the warps share each head's dependent load-and-add chain.
 constexpr int kMaxSplits = 64;
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -504,30 +506,35 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float
   }
 }
 
-template <int G>
-__global__ void __launch_bounds__(64 * G)
+template <int G, int SP>
+__global__ void __launch_bounds__(64 * G * SP)
     mla_combine_kernel(const __nv_bfloat16* __restrict__ ws_o, const float* __restrict__ ws_ml, int H,
                        int n_splits, void* out, int out_bf16, float* lse) {
+  static_assert(G == 1 || SP == 1, "several heads or several parts per head, not both");
   __shared__ float s_w[G][kMaxSplits];
   __shared__ float s_ml[G][2];
+  __shared__ float4 s_part[SP > 1 ? (SP - 1) * 64 * 2 : 1];  // parts 1.. of each column group
   grid_dependency_wait();  // partials come from the previous kernel
   allow_dependents_launch();
   const int groups = (H + G - 1) / G;  // head groups per row
   const int64_t r = blockIdx.x / groups;
-  const int g = threadIdx.x >> 6;      // head of the group
+  const int g = SP > 1 ? 0 : threadIdx.x >> 6;   // head of the group
+  const int part = SP > 1 ? threadIdx.x >> 6 : 0;  // this thread's splits: part, part + SP, ...
   const int64_t h = (int64_t)(blockIdx.x % groups) * G + g;
-  const bool live = h < H;             // uniform over the head's two warps
+  const bool live = h < H;             // uniform over the head's warps
   const int64_t rh = r * H + h;
   const int c8 = threadIdx.x & 63;  // eight columns: 8*c8 .. 8*c8+7
   const uint4* base = reinterpret_cast<const uint4*>(ws_o + (r * n_splits * H + (live ? h : 0)) * kDV) + c8;
-  const int64_t stride = (int64_t)H * kDV / 8;  // uint4 between consecutive splits
+  const int64_t stride = (int64_t)H * kDV / 8 * SP;  // uint4 between this thread's consecutive splits
+  const int n_mine = (n_splits - part + SP - 1) / SP;
   // splits whose loads are in flight at once (registers: 512 threads at G = 8)
-  constexpr int NB = G == 1 ? 32 : 16;
+  constexpr int NB = G == 1 && SP == 1 ? 32 : 16;
   uint4 o[NB];
+  const uint4* mine = base + (int64_t)part * (stride / SP);
 #pragma unroll
   for (int s = 0; s < NB; ++s)
-    if (live && s < n_splits) o[s] = __ldg(base + s * stride);
-  if (live && c8 < 32) {
+    if (live && s < n_mine) o[s] = __ldg(mine + s * stride);
+  if (live && part == 0 && c8 < 32) {
     const int s0 = c8, s1 = c8 + 32;
     float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
     if (s0 < n_splits) {
@@ -556,19 +563,41 @@ __global__ void __launch_bounds__(64 * G)
     }
   }
   __syncthreads();
-  if (!live) return;  // no barrier below
-  const float M = s_ml[g][0], L = s_ml[g][1];
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int sb = 0; sb < n_splits; sb += NB) {
-    if (sb > 0) {  // the next group of splits
+  if (live) {
+    for (int sb = 0; sb < n_mine; sb += NB) {
+      if (sb > 0) {  // the next group of this thread's splits
+#pragma unroll
+        for (int s = 0; s < NB; ++s)
+          if (sb + s < n_mine) o[s] = __ldg(mine + (sb + s) * stride);
+      }
 #pragma unroll
       for (int s = 0; s < NB; ++s)
-        if (sb + s < n_splits) o[s] = __ldg(base + (sb + s) * stride);
+        if (sb + s < n_mine) acc_bf16x8(acc, o[s], s_w[g][part + SP * (sb + s)]);
     }
-#pragma unroll
-    for (int s = 0; s < NB; ++s)
-      if (sb + s < n_splits) acc_bf16x8(acc, o[s], s_w[g][sb + s]);
   }
+  if constexpr (SP > 1) {
+    if (part > 0) {
+      s_part[((part - 1) * 64 + c8) * 2] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      s_part[((part - 1) * 64 + c8) * 2 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+    __syncthreads();
+    if (part > 0) return;  // no barrier below
+#pragma unroll
+    for (int q = 0; q < SP - 1; ++q) {
+      const float4 a = s_part[(q * 64 + c8) * 2], b = s_part[(q * 64 + c8) * 2 + 1];
+      acc[0] += a.x;
+      acc[1] += a.y;
+      acc[2] += a.z;
+      acc[3] += a.w;
+      acc[4] += b.x;
+      acc[5] += b.y;
+      acc[6] += b.z;
+      acc[7] += b.w;
+    }
+  }
+  if (!live) return;
+  const float M = s_ml[g][0], L = s_ml[g][1];
   const float inv = L > 0.f ? 1.f / L : 0.f;
   if (out_bf16) {
     uint32_t w4[4];
@@ -600,11 +629,16 @@ cudaError_t launch_combine(const MlaParams& p, int64_t n_rows, int H, cudaStream
   const dim3 grid((unsigned)(n_rows * ((H + G - 1) / G)));
   const __nv_bfloat16* o = p.ws_o;
   const float* ml = p.ws_ml;
+  const int ns = p.n_splits;
   switch (G) {
-    case 1: return launch_pdl(mla_combine_kernel<1>, grid, dim3(64), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
-    case 2: return launch_pdl(mla_combine_kernel<2>, grid, dim3(128), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
-    case 4: return launch_pdl(mla_combine_kernel<4>, grid, dim3(256), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
-    default: return launch_pdl(mla_combine_kernel<8>, grid, dim3(512), 0, stream, o, ml, H, p.n_splits, p.out, p.out_bf16, p.lse);
+    case 1:
+      // one head per CTA: with eight or more splits, four parts per head
+      if (ns >= 8)
+        return launch_pdl(mla_combine_kernel<1, 4>, grid, dim3(256), 0, stream, o, ml, H, ns, p.out, p.out_bf16, p.lse);
+      return launch_pdl(mla_combine_kernel<1, 1>, grid, dim3(64), 0, stream, o, ml, H, ns, p.out, p.out_bf16, p.lse);
+    case 2: return launch_pdl(mla_combine_kernel<2, 1>, grid, dim3(128), 0, stream, o, ml, H, ns, p.out, p.out_bf16, p.lse);
+    case 4: return launch_pdl(mla_combine_kernel<4, 1>, grid, dim3(256), 0, stream, o, ml, H, ns, p.out, p.out_bf16, p.lse);
+    default: return launch_pdl(mla_combine_kernel<8, 1>, grid, dim3(512), 0, stream, o, ml, H, ns, p.out, p.out_bf16, p.lse);
   }
 }
 

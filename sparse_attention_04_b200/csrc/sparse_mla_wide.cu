@@ -521,17 +521,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                       mbar_wait(pv_done((n_my - 1) & 1), ((n_my - 1) >> 1) & 1, abort, p.wait_limit_ns));
     // Every MMA has completed, so the query blocks and key stages are free:
     // the 128 x 256 result is staged there as 128-byte-swizzled boxes of 32
-    // fp32 (or 64 bf16) columns, one thread per head row, and written by a
-    // few TMA tensor stores (the output's tensor map has one box per block).
+    // fp32 (or 64 bf16) columns, one thread per head row, and written by TMA
+    // tensor stores (the output's tensor map has one box per block).  Each
+    // 64-column slice is stored as soon as it is staged, so the copy of one
+    // overlaps the staging of the next.
     const bool final_out = p.n_splits == 1;
     const bool as_bf16 = !final_out || p.out_bf16;  // partials are bf16 too
-    if (ok) {
-      tc_fence_after();
-      const float mul = final_out ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
-      uint8_t* stage = smem;
-      const int sw = h & 7;
+    const int y_out = final_out ? r * p.H : (r * p.n_splits + sp) * p.H;
+    if (ok) tc_fence_after();
+    const float mul = final_out ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
+    uint8_t* stage = smem;
+    const int sw = h & 7;
 #pragma unroll 1
-      for (int cb2 = 0; cb2 < 8; cb2 += 2) {
+    for (int cb2 = 0; cb2 < 8; cb2 += 2) {
+      if (ok) {
         uint32_t ovp[2][32];
         tmem_ld32(lane_addr + 32 * cb2, ovp[0]);
         tmem_ld32(lane_addr + 32 * cb2 + 32, ovp[1]);
@@ -563,15 +566,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                               __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
           }
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-    }
-    named_barrier_sync(1, 128);  // every epilogue warp, whatever its wait outcome
-    if (threadIdx.x == 0 && !*abort) {
-      const int nblk = as_bf16 ? 4 : 8, colw = as_bf16 ? 64 : 32;
-      const int y = final_out ? r * p.H : (r * p.n_splits + sp) * p.H;
-      for (int bk = 0; bk < nblk; ++bk) tma_store_2d(&tm_out, sbase + bk * kStageBlock, 256 * v + colw * bk, y);
-      bulk_commit();
+      named_barrier_sync(1, 128);  // every epilogue warp, whatever its wait outcome
+      if (threadIdx.x == 0 && !*abort) {
+        if (as_bf16) {
+          tma_store_2d(&tm_out, sbase + (cb2 >> 1) * kStageBlock, 256 * v + 32 * cb2, y_out);
+        } else {
+          tma_store_2d(&tm_out, sbase + cb2 * kStageBlock, 256 * v + 32 * cb2, y_out);
+          tma_store_2d(&tm_out, sbase + (cb2 + 1) * kStageBlock, 256 * v + 32 * (cb2 + 1), y_out);
+        }
+        bulk_commit();
+      }
     }
     if (ok && h < p.H && v == 0) {
       const int64_t rh = (int64_t)r * p.H + h;
