@@ -691,8 +691,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Every MMA has completed, so the value ring is free: the 128 x 512
       // result is staged there as 128-byte-swizzled boxes of 32 fp32 (or 64
       // bf16) columns, one thread per head row, and written by TMA tensor
-      // stores (the output's tensor map has one box per block).  fp32 output
-      // goes in two halves of 256 columns.
+      // stores (the output's tensor map has one box per block), each 64
+      // columns as soon as they are staged.  fp32 output goes in two halves
+      // of 256 columns.
       const bool final_out = p.n_splits == 1;
       const bool as_bf16 = !final_out || p.out_bf16;  // partials are bf16 too
       const float mul = final_out ? (l_row > 0.f ? 1.f / l_row : 0.f) : 1.f;
@@ -700,11 +701,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int y = final_out ? r * p.H : (r * p.n_splits + sp) * p.H;
       const int n_pass = as_bf16 ? 1 : 2;
       for (int pass = 0; pass < n_pass; ++pass) {
-        if (ok) {
-          tc_fence_after();
-          const int cb_lo = as_bf16 ? 0 : 8 * pass, cb_hi = as_bf16 ? 16 : 8 * pass + 8;
+        if (ok) tc_fence_after();
+        const int cb_lo = as_bf16 ? 0 : 8 * pass, cb_hi = as_bf16 ? 16 : 8 * pass + 8;
 #pragma unroll 1
-          for (int cb2 = cb_lo; cb2 < cb_hi; cb2 += 2) {
+        for (int cb2 = cb_lo; cb2 < cb_hi; cb2 += 2) {
+          if (ok) {
             uint32_t ovp[2][32];
             tmem_ld32(lane_addr + 32 * cb2, ovp[0]);
             tmem_ld32(lane_addr + 32 * cb2 + 32, ovp[1]);
@@ -736,19 +737,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                   __uint_as_float(ov[4 * q4 + 2]) * mul, __uint_as_float(ov[4 * q4 + 3]) * mul);
               }
             }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
-        }
-        named_barrier_sync(1, 128);  // every epilogue warp, whatever its wait outcome
-        if (threadIdx.x == 0 && !*abort) {
-          if (as_bf16) {
-            for (int bk = 0; bk < 8; ++bk) tma_store_2d(&tm_out, sbase + bk * kStageBlock, 64 * bk, y);
-          } else {
-            for (int bk = 0; bk < 8; ++bk) tma_store_2d(&tm_out, sbase + bk * kStageBlock, 256 * pass + 32 * bk, y);
+          named_barrier_sync(1, 128);  // every epilogue warp, whatever its wait outcome
+          if (threadIdx.x == 0 && !*abort) {
+            if (as_bf16) {
+              tma_store_2d(&tm_out, sbase + (cb2 >> 1) * kStageBlock, 32 * cb2, y);
+            } else {
+              tma_store_2d(&tm_out, sbase + (cb2 - cb_lo) * kStageBlock, 32 * cb2, y);
+              tma_store_2d(&tm_out, sbase + (cb2 + 1 - cb_lo) * kStageBlock, 32 * (cb2 + 1), y);
+            }
+            bulk_commit();
           }
-          bulk_commit();
-          bulk_wait_read();  // the staged boxes stay valid until read
         }
+        if (threadIdx.x == 0 && !*abort) bulk_wait_read();  // the staged boxes stay valid until read
         named_barrier_sync(1, 128);
       }
       if (ok && h < p.H) {

@@ -4,6 +4,7 @@ device-side timeout path.
   - the e4m3 indexer with T > 1 (causal prefill rows of ragged sequences);
   - the attention at head counts other than 16 and 128, both output types;
   - the combine with several heads per CTA (a partly filled last group);
+  - the pair kernel with fp32 output;
   - split rows on a workspace that starts zero, all ones or random, reused;
   - a short-context decode step whose query was written by the kernel copy
     just before it on the same stream;
@@ -124,6 +125,18 @@ def test_short_context_head_counts(cuda_device, H):
     for b, E in enumerate(sub.end_pos):
         full[b, :E] = torch.arange(E, dtype=torch.int32)
     check_mla(res.out.reshape(2, H, -1), res.lse.reshape(2, H), full, sub, [0, 1])
+
+
+# ------------------------------------------------------------------ pair kernel, fp32 output
+
+def test_pair_kernel_fp32_output(cuda_device):
+    """160 causal prefill rows, k = 2048: enough 128-key chunks for the
+    pair kernel (QK CTA + PV CTA), one unit per row, and fp32 output, which
+    its epilogue writes in two 256-column passes through the value ring."""
+    from test_parity_gpu import run_and_check as rc
+    wl = dsa_inputs.custom("pair_f32", B=1, T=160, end_pos=None, topk=2048, H=128, out_dtype="f32",
+                           scale=192 ** -0.5, seed=111, end_pos_range=(1, 1))
+    rc(wl, cuda_device, end_pos=[400], rows=[0, 1, 2, 79, 158, 159])
 
 
 # ------------------------------------------------------------------ split rows on a reused workspace
