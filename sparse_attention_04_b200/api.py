@@ -68,15 +68,16 @@ class HostDecodeStep:
         -> dsa_topk -> dsa_sparse_mla -> copy kernel (out)
 
     and on a side stream the transfer of q, the largest input, which only the
-    attention reads: it crosses PCIe while the indexer and the selection run,
-    and the attention waits for it.  Up to Q_KERNEL_COPY_MAX bytes a copy
-    kernel moves q (it finishes within the indexer and leaves the chain free
-    of copy-engine hand-offs, each of which costs several microseconds);
-    above that the copy engine does, so that a long transfer holds no SM
-    while the indexer and the selection want them all.  When every end_pos
-    <= k the attention-only form of dsa_decode_step runs after that wait
-    instead.  Each call starts after everything issued before it on the
-    stream."""
+    attention reads; the attention waits for it.  Up to Q_KERNEL_COPY_MAX
+    bytes a copy kernel moves q, launched once the indexer has finished: it
+    crosses PCIe while the selection runs on a few SMs.  Started with the
+    step, its CTAs took registers the indexer's CTAs needed on their SMs and
+    held those CTAs back (decode 32K: 38.8 against 37.5 us per step, fp8
+    B=4: 78.8 against 71.4 us).  A larger q goes by the copy engine from the
+    start of the step, so that a long transfer overlaps the indexer as well
+    and holds no SM.  When every end_pos <= k the attention-only form of
+    dsa_decode_step runs after the transfer instead.  Each call starts after
+    everything issued before it on the stream."""
 
     Q_KERNEL_COPY_MAX = 1 << 20
 
@@ -114,27 +115,36 @@ class HostDecodeStep:
         self.h2d_bytes = tot + self.host_q.numel() * 2
         self.d2h_bytes = self.host_out.numel() * self.host_out.element_size()
 
-    def __call__(self, k_idx, k_scale, kv, offsets, kv_rows, scale):
-        st, B = self.step, self.B
-        cur = torch.cuda.current_stream()
+    def _copy_q(self, cur):
+        """q's transfer on the side stream, after everything issued so far on `cur`."""
         self._side.wait_stream(cur)
         with torch.cuda.stream(self._side):
             if self.host_q.numel() * 2 <= self.Q_KERNEL_COPY_MAX:
                 _lib.copy_host_to_device(self._q, self.host_q)
             else:
                 self._q.copy_(self.host_q, non_blocking=True)
+
+    def __call__(self, k_idx, k_scale, kv, offsets, kv_rows, scale):
+        st, B = self.step, self.B
+        cur = torch.cuda.current_stream()
+        q_by_kernel = self.host_q.numel() * 2 <= self.Q_KERNEL_COPY_MAX
+        short = self.max_end_pos <= self.k
+        if short or not q_by_kernel:
+            self._copy_q(cur)
         _lib.copy_host_to_device(self._small, self.host_small)
         _lib.cache_append(self._k_new, self._kv_new, offsets, B, 1, k_idx, k_scale, kv, kv_rows, status=st.status)
         q_idx, w = self._q_idx, self._w
         if self.fp8:
             _lib.quantize_queries(q_idx, w, B, self._q8, self._w8)
             q_idx, w = self._q8, self._w8
-        if self.max_end_pos <= self.k:
+        if short:
             cur.wait_stream(self._side)
             st(q_idx, w, k_idx, k_scale, self._q, kv, offsets, kv_rows, scale)
         else:
             _lib.indexer_scores(q_idx, w, k_idx, k_scale, offsets, B, 1, kv_rows, st.scores, st.ld,
                                 status=st.status)
+            if q_by_kernel:
+                self._copy_q(cur)  # crosses PCIe beside the selection
             _lib.topk(st.scores, st.ld, offsets, B, 1, self.k, st.indices, status=st.status)
             cur.wait_stream(self._side)
             _lib.sparse_mla(self._q, kv, offsets, st.indices, B, 1, self.H, self.k, scale, kv_rows, st.out,
