@@ -67,18 +67,25 @@ class HostDecodeStep:
         -> [dsa_quantize_queries for e4m3 keys] -> dsa_indexer_scores
         -> dsa_topk -> dsa_sparse_mla -> copy kernel (out)
 
-    and on a side stream the transfer of q, the largest input, which only the
-    attention reads; the attention waits for it.  Up to Q_KERNEL_COPY_MAX
-    bytes a copy kernel moves q, launched once the indexer has finished: it
-    crosses PCIe while the selection runs on a few SMs.  Started with the
-    step, its CTAs took registers the indexer's CTAs needed on their SMs and
-    held those CTAs back (decode 32K: 38.8 against 37.5 us per step, fp8
-    B=4: 78.8 against 71.4 us).  A larger q goes by the copy engine from the
-    start of the step, so that a long transfer overlaps the indexer as well
-    and holds no SM.  When every end_pos <= k the attention-only form of
-    dsa_decode_step runs after the transfer instead.  Each call starts after
-    everything issued before it on the stream."""
+    How q, the largest input, crosses PCIe depends on its size (measured on
+    B200, microseconds per host-fed step):
+      - up to Q_WITH_INPUTS_MAX bytes (one 128-head row): in the same copy
+        kernel as the small inputs, so that the whole dsa_decode_step follows
+        with q complete and the attention loads its query tile before the
+        selection ends (decode 32K: 36.3 against 37.5 with the side stream);
+      - up to Q_KERNEL_COPY_MAX bytes: on a side stream, by a copy kernel
+        launched once the indexer has finished, so it crosses PCIe while the
+        selection runs on a few SMs; the attention waits for it.  Started with
+        the step, its CTAs took registers that the indexer's CTAs needed and
+        held them back (fp8 B=4: 78.8 against 71.4; in the first copy 78.1);
+      - above that: by the copy engine on the side stream from the start of
+        the step, so that a long transfer overlaps the indexer too and holds
+        no SM.
+    When every end_pos <= k the attention-only form of dsa_decode_step runs
+    once q is in.  Each call starts after everything issued before it on the
+    stream."""
 
+    Q_WITH_INPUTS_MAX = 1 << 18
     Q_KERNEL_COPY_MAX = 1 << 20
 
     def __init__(self, B: int, max_end_pos: int, k: int, H: int, idx_dtype: str = "bf16",
@@ -87,9 +94,14 @@ class HostDecodeStep:
         self.step = DecodeStep(B, max_end_pos, k, H, out_dtype, dev)
         self.B, self.max_end_pos, self.k, self.H = B, max_end_pos, k, H
         self.fp8 = idx_dtype == "e4m3"
-        # one pinned staging buffer for the small inputs, 256-byte aligned sections
+        # one pinned staging buffer for the small inputs (and q, when it is
+        # small enough to travel with them), 256-byte aligned sections
+        q_bytes = B * H * 576 * 2
+        self.q_with_inputs = q_bytes <= self.Q_WITH_INPUTS_MAX
         spec = [(torch.bfloat16, (B, 1, 64, 128)), (torch.float32, (B, 1, 64)),
                 (torch.bfloat16, (B, 1, 128)), (torch.bfloat16, (B, 1, 576))]
+        if self.q_with_inputs:
+            spec.append((torch.bfloat16, (B, 1, H, 576)))
         sizes = [math.prod(shape) * torch.empty((), dtype=dt).element_size() for dt, shape in spec]
         offs, tot = [], 0
         for sz in sizes:
@@ -101,10 +113,14 @@ class HostDecodeStep:
         def views(buf):
             return [buf[o:o + n].view(dt).view(*shape) for o, n, (dt, shape) in zip(offs, sizes, spec)]
 
-        self.host_q_idx, self.host_w, self.host_k_new, self.host_kv_new = views(self.host_small)
-        self._q_idx, self._w, self._k_new, self._kv_new = views(self._small)
-        self.host_q = torch.zeros((B, 1, H, 576), dtype=torch.bfloat16, pin_memory=True)
-        self._q = torch.empty((B, 1, H, 576), dtype=torch.bfloat16, device=dev)
+        hv, dv = views(self.host_small), views(self._small)
+        self.host_q_idx, self.host_w, self.host_k_new, self.host_kv_new = hv[:4]
+        self._q_idx, self._w, self._k_new, self._kv_new = dv[:4]
+        if self.q_with_inputs:
+            self.host_q, self._q = hv[4], dv[4]
+        else:
+            self.host_q = torch.zeros((B, 1, H, 576), dtype=torch.bfloat16, pin_memory=True)
+            self._q = torch.empty((B, 1, H, 576), dtype=torch.bfloat16, device=dev)
         self.host_out = torch.zeros(tuple(self.step.out.shape), dtype=out_dtype, pin_memory=True)
         if self.fp8:
             self._q8 = torch.empty((B, 1, 64, 128), dtype=torch.uint8, device=dev)
@@ -112,7 +128,7 @@ class HostDecodeStep:
         m_off = _lib.decode_step_workspace_layout(B, max_end_pos, k, H)[3]
         self._ws_mla = self.step.workspace[m_off:]
         self._side = torch.cuda.Stream(dev)
-        self.h2d_bytes = tot + self.host_q.numel() * 2
+        self.h2d_bytes = tot + (0 if self.q_with_inputs else self.host_q.numel() * 2)
         self.d2h_bytes = self.host_out.numel() * self.host_out.element_size()
 
     def _copy_q(self, cur):
@@ -129,7 +145,7 @@ class HostDecodeStep:
         cur = torch.cuda.current_stream()
         q_by_kernel = self.host_q.numel() * 2 <= self.Q_KERNEL_COPY_MAX
         short = self.max_end_pos <= self.k
-        if short or not q_by_kernel:
+        if not self.q_with_inputs and (short or not q_by_kernel):
             self._copy_q(cur)
         _lib.copy_host_to_device(self._small, self.host_small)
         _lib.cache_append(self._k_new, self._kv_new, offsets, B, 1, k_idx, k_scale, kv, kv_rows, status=st.status)
@@ -137,7 +153,10 @@ class HostDecodeStep:
         if self.fp8:
             _lib.quantize_queries(q_idx, w, B, self._q8, self._w8)
             q_idx, w = self._q8, self._w8
-        if short:
+        if self.q_with_inputs:
+            # q is complete before the step's first kernel: the fused step
+            st(q_idx, w, k_idx, k_scale, self._q, kv, offsets, kv_rows, scale)
+        elif short:
             cur.wait_stream(self._side)
             st(q_idx, w, k_idx, k_scale, self._q, kv, offsets, kv_rows, scale)
         else:

@@ -24,9 +24,12 @@ def _fill_host(hs, B, H, seed):
     hs.host_kv_new.copy_(torch.randn(B, 1, 576, generator=g).to(torch.bfloat16))
 
 
-# q of the last case is above HostDecodeStep.Q_KERNEL_COPY_MAX: the copy engine moves it
+# How q crosses PCIe depends on its size: with the small inputs (the first
+# three cases), by a side-stream copy kernel after the indexer (the fourth,
+# 295 KB), by the copy engine (the last, above HostDecodeStep.Q_KERNEL_COPY_MAX)
 @pytest.mark.parametrize("idx_dtype,eps,k,H", [("bf16", [3000, 5000, 1500], 2048, 16), ("e4m3", [700, 1200], 256, 16),
                                                ("bf16", [100, 2048, 1], 2048, 16),
+                                               ("bf16", [3000, 2500], 2048, 128),
                                                ("bf16", [900, 1300, 600, 1000, 700, 2000, 650, 1100], 512, 128)])
 def test_host_step_matches_device_path_and_oracle(cuda_device, idx_dtype, eps, k, H):
     from sparse_attention_04_b200 import _lib, api
@@ -37,7 +40,9 @@ def test_host_step_matches_device_path_and_oracle(cuda_device, idx_dtype, eps, k
     k2, kv2 = inp.k_idx.clone(), inp.kv.clone()
     ks2 = None if inp.k_scale is None else inp.k_scale.clone()
     hs = api.HostDecodeStep(B, max(eps), k, H, idx_dtype, torch.bfloat16, cuda_device)
-    assert (B * H * 576 * 2 > hs.Q_KERNEL_COPY_MAX) == (H == 128)
+    q_bytes = B * H * 576 * 2  # the path the step takes for q, as the cases above intend
+    path = "inputs" if q_bytes <= hs.Q_WITH_INPUTS_MAX else "kernel" if q_bytes <= hs.Q_KERNEL_COPY_MAX else "engine"
+    assert path == ("inputs" if H == 16 else "kernel" if B == 2 else "engine") and hs.q_with_inputs == (path == "inputs")
     for seed in (1, 2):  # two calls: the second must see the refilled host inputs
         _fill_host(hs, B, H, 70 + seed)
         out = hs(inp.k_idx, inp.k_scale, inp.kv, inp.offsets, inp.rows, wl.scale)
@@ -79,12 +84,14 @@ def test_host_step_matches_device_path_and_oracle(cuda_device, idx_dtype, eps, k
         check_mla(out.reshape(B, H, -1), hs.step.lse.reshape(B, H), idx, sub, list(range(B)))
 
 
-def test_host_step_in_a_cuda_graph(cuda_device):
+@pytest.mark.parametrize("H", [16, 128])
+def test_host_step_in_a_cuda_graph(cuda_device, H):
     """Captured once, replayed with the host inputs refilled between
     replays: each replay's output matches an eager host-fed step on the same
-    inputs and caches."""
+    inputs and caches.  H = 16: q travels with the small inputs; H = 128
+    (295 KB): by a side-stream copy kernel after the indexer."""
     from sparse_attention_04_b200 import api
-    B, H, k = 2, 16, 512
+    B, k = 2, 512
     eps = [9000, 3000]
     wl = dsa_inputs.custom("host_graph", B=B, end_pos=None, topk=k, H=H, out_dtype="bf16", seed=91,
                            end_pos_range=(1, 1))
